@@ -1,0 +1,493 @@
+#!/usr/bin/env python
+"""Benchmark of the exact attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one forward over one batch of the main workload (default: the
+varlen causal GQA 32/8 D=128 workload with a 256-wide relative bias, 4
+sequences of seeded lengths in [512, 4096]).  Rank 0 prints ONE JSON line with
+the throughput in TFLOP/s (4 * q_len * k_len * D * Hq per sequence, halved for
+causal), the roofline of the kernel, the CPU oracle baseline, an end-to-end
+figure through host buffers, the SM clocks seen while timing, and the other
+workloads measured the same way ("workloads").
+
+Multi-GPU (launched by torchrun): every rank runs its own copy of the workload
+(independent problems, no data-path collective: weak scaling); the time is the
+maximum over ranks of the device-measured time.
+
+``--impl reference`` times the CPU fp64 oracle instead (rank 0 only), on a
+bounded sample of rows of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd TFLOP/s & % of BF16 tensor peak; split-KV decode HBM GB/s"
+MAIN = "varlen_gqa_bias"
+EXTRAS = ["dense_257", "video_dit_20480", "encoder_d256_seqused", "decode_splitkv"]
+DESCR = {
+    "dense_257": "dense non-causal MHA B=1 S=257 H=8 D=128 bf16",
+    "varlen_gqa_bias": "varlen causal GQA 32/8 D=128, 4 seqs U[512,4096] (seeded), rel_bias R=256 bf16",
+    "video_dit_20480": "dense non-causal MHA B=1 S=20480 H=56 D=128 bf16",
+    "encoder_d256_seqused": "dense GQA 8/1 D=256 B=2 Sq=1024 Sk=1024 seqused_k=968 bf16",
+    "decode_splitkv": "split-KV decode B=8 Sq=1 Sk=131072 Hq=32 Hkv=8 D=128 bf16",
+}
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=MAIN)
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--splits", type=int, default=0, help="split-KV count (0 = auto)")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# peaks, profiles, clocks
+# ---------------------------------------------------------------------------
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"bf16_tflops": float(d["bf16_tflops"]), "hbm_gbs": float(d["hbm_gbs"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return dict(FALLBACK_PEAKS, bf16_tflops_sustained=FALLBACK_PEAKS["bf16_tflops"],
+                    source="fallback")
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "exact_attention_forward_flash_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the main kernel from the committed ncu
+    summary, if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", f"fa_fwd_{workload}.ncu.txt")
+    try:
+        kv = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line:
+                    a, b = line.split(":", 1)
+                    kv[a.strip()] = b.strip()
+        if kv.get("kernel_source_sha256") != kernel_source_hash():
+            return None
+        return float(kv["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML in a thread."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.002):
+        self.samples, self.reasons = [], 0
+        self.period = period_s
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                try:
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except AttributeError:
+                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.reasons |= int(r)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# workloads on the device
+# ---------------------------------------------------------------------------
+BIG = {"video_dit_20480", "decode_splitkv"}
+
+
+def build_problem(name: str, device):
+    import fa_inputs
+    if name in BIG:
+        return fa_inputs.make(name, device=device)
+    return fa_inputs.make(name).to(device)
+
+
+class Runner:
+    """Preallocated outputs and one call per step through the C ABI."""
+
+    def __init__(self, p, splits: int = 0):
+        import torch
+        import exact_attention_forward_flash_b200 as fa
+        self.fa, self.p = fa, p
+        self.out = torch.empty_like(p.q)
+        if p.layout == "dense":
+            self.lse = torch.empty((p.B, p.Hq, p.q.shape[1]), dtype=torch.float32, device=p.q.device)
+        else:
+            self.lse = torch.empty((p.Hq, p.q.shape[0]), dtype=torch.float32, device=p.q.device)
+        self.ws = None
+        self.launches = 1
+        if p.splitkv:
+            B, Sq, Hq, D = p.q.shape
+            Sk, Hkv = p.k.shape[1], p.k.shape[2]
+            n_sms = torch.cuda.get_device_properties(p.q.device).multi_processor_count
+            self.ns = splits or fa.splitkv_default_splits(B, Sq, Sk, Hq, Hkv, D, n_sms)
+            nbytes = fa.splitkv_workspace_bytes(B, Sq, Hq, D, self.ns)
+            self.ws = torch.empty(nbytes, dtype=torch.uint8, device=p.q.device)
+            self.launches = 2
+
+    def __call__(self, q=None, k=None, v=None, rel_bias=None, cu=None):
+        p, fa = self.p, self.fa
+        q = p.q if q is None else q
+        k = p.k if k is None else k
+        v = p.v if v is None else v
+        rb = p.rel_bias if rel_bias is None else rel_bias
+        if p.splitkv:
+            fa.fa_fwd_splitkv(q, k, v, num_splits=self.ns, causal=p.causal,
+                              softmax_scale=p.softmax_scale, seqused_k=p.seqused_k,
+                              rel_bias=rb, out=self.out, lse=self.lse, workspace=self.ws)
+        elif p.layout == "dense":
+            fa.fa_fwd(q, k, v, causal=p.causal, softmax_scale=p.softmax_scale,
+                      seqused_k=p.seqused_k, rel_bias=rb, out=self.out, lse=self.lse)
+        else:
+            cq, ck = (p.cu_seqlens_q, p.cu_seqlens_k) if cu is None else cu
+            fa.fa_fwd_varlen(q, k, v, cq, ck, p.max_seqlen_q, p.max_seqlen_k,
+                             seqused_k=p.seqused_k, causal=p.causal,
+                             softmax_scale=p.softmax_scale, rel_bias=rb, out=self.out,
+                             lse=self.lse)
+
+
+def time_steps(step, steps: int, warmup: int, dist_on: bool, device_index: int):
+    """W untimed steps, then K steps between barrier + synchronize; returns
+    (total ms over K, mean per-step ms from per-step events, clocks)."""
+    import torch
+    import torch.distributed as dist
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist_on:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(device_index) as clk:
+        t0.record()
+        for a, b in evs:
+            a.record()
+            step()
+            b.record()
+        t1.record()
+        torch.cuda.synchronize()
+    if dist_on:
+        dist.barrier()
+    total = t0.elapsed_time(t1)
+    per = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    return total, per, clk.summary()
+
+
+def max_over_ranks(x: float, dist_on: bool) -> float:
+    if not dist_on:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def roofline(p, per_launch_ms: float, peaks, traffic):
+    if p.splitkv:
+        achieved = p.hbm_bytes() / (per_launch_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "peak_source": peaks["source"]}
+    achieved = p.flops() / (per_launch_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    return {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "peak_source": peaks["source"] + " (burst)"}
+
+
+def workload_value(p, ms):
+    if p.splitkv:
+        return p.hbm_bytes() / (ms * 1e-3) / 1e9, "GB/s"
+    return p.flops() / (ms * 1e-3) / 1e12, "TFLOP/s"
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded row sample)
+# ---------------------------------------------------------------------------
+def oracle_rows_sample(p, n_rows: int, seed: int = 0):
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    lens = p.seq_lens()
+    B = len(lens)
+    rows, flops = [], 0.0
+    for _ in range(n_rows):
+        b = int(rng.integers(B))
+        ql, kl = lens[b]
+        while ql == 0:
+            b = int(rng.integers(B))
+            ql, kl = lens[b]
+        i = int(rng.integers(ql))
+        h = int(rng.integers(p.Hq))
+        keys = min(kl, i + (kl - ql) + 1) if p.causal else kl
+        flops += 4.0 * p.D * max(keys, 0)
+        rows.append((b, h, i))
+    return np.array(rows, dtype=np.int32), flops
+
+
+def time_oracle(p_cpu, target_s: float):
+    import oracle
+    kw = dict(causal=p_cpu.causal, softmax_scale=p_cpu.softmax_scale,
+              seqused_k=p_cpu.seqused_k, rel_bias=p_cpu.rel_bias)
+    if p_cpu.layout == "varlen":
+        kw.update(cu_seqlens_q=p_cpu.cu_seqlens_q, cu_seqlens_k=p_cpu.cu_seqlens_k)
+    n = 64
+    while True:
+        rows, flops = oracle_rows_sample(p_cpu, n)
+        t = time.perf_counter()
+        oracle.attention_rows(p_cpu.q, p_cpu.k, p_cpu.v, rows, **kw)
+        dt = time.perf_counter() - t
+        if dt >= 0.5 * target_s or n >= 1 << 22:
+            return flops / dt / 1e12, dt, n
+        n = int(n * min(64.0, max(2.0, target_s / max(dt, 1e-3))))
+
+
+# ---------------------------------------------------------------------------
+def main():
+    a = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if a.impl == "reference":
+        if rank != 0:
+            return 0
+        return run_reference(a, world)
+
+    import torch
+    import torch.distributed as dist
+    import exact_attention_forward_flash_b200 as fa
+    fa.load_library()
+    dist_on = world > 1
+    torch.cuda.set_device(local)
+    if dist_on:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+
+    # ---- main workload, device-resident inputs
+    import fa_inputs
+    p_cpu = fa_inputs.make(a.workload) if a.workload not in BIG else None
+    p = build_problem(a.workload, dev)
+    run = Runner(p, a.splits)
+    total_ms, per_ms, clocks = time_steps(run, a.steps, a.warmup, dist_on, local)
+    total_ms = max_over_ranks(total_ms, dist_on)
+    ms_step = total_ms / a.steps
+    value = world * workload_value(p, ms_step)[0]
+    unit = workload_value(p, ms_step)[1]
+    traffic = profiled_traffic(a.workload)
+    roof = roofline(p, per_ms, peaks, traffic)
+
+    # ---- end to end: pinned host inputs -> device -> library -> host outputs
+    e2e = None
+    if not p.splitkv and p_cpu is not None:
+        hq, hk, hv = (p_cpu.q.pin_memory(), p_cpu.k.pin_memory(), p_cpu.v.pin_memory())
+        hb = p_cpu.rel_bias.pin_memory() if p_cpu.rel_bias is not None else None
+        hcu = (p_cpu.cu_seqlens_q.pin_memory(), p_cpu.cu_seqlens_k.pin_memory()) \
+            if p_cpu.cu_seqlens_q is not None else None
+        dq, dk, dv = torch.empty_like(p.q), torch.empty_like(p.k), torch.empty_like(p.v)
+        db = torch.empty_like(p.rel_bias) if hb is not None else None
+        dcu = (torch.empty_like(p.cu_seqlens_q), torch.empty_like(p.cu_seqlens_k)) if hcu else None
+        ho = torch.empty(p.q.shape, dtype=p.q.dtype).pin_memory()
+        hl = torch.empty(run.lse.shape, dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            if db is not None:
+                db.copy_(hb, non_blocking=True)
+            if dcu is not None:
+                dcu[0].copy_(hcu[0], non_blocking=True)
+                dcu[1].copy_(hcu[1], non_blocking=True)
+            run(dq, dk, dv, db, dcu)
+            ho.copy_(run.out, non_blocking=True)
+            hl.copy_(run.lse, non_blocking=True)
+
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv) + ((hb,) if hb is not None else ()) + (hcu or ()))
+        d2h = ho.numel() * ho.element_size() + hl.numel() * 4
+        e_steps = max(3, min(a.steps, 20))
+        e_total, _, _ = time_steps(e2e_step, e_steps, 2, dist_on, local)
+        e_total = max_over_ranks(e_total, dist_on)
+        ev = world * workload_value(p, e_total / e_steps)[0]
+        e2e = {"value": round(ev, 3), "unit": unit, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e_total / e_steps, 4)}
+
+    # ---- the other workloads, same protocol (rank 0 reports its own)
+    extras = {}
+    if not a.no_extras:
+        for name in EXTRAS:
+            if name == a.workload:
+                continue
+            q = build_problem(name, dev)
+            r = Runner(q, a.splits)
+            k_steps = max(5, min(a.steps, 30))
+            tt, pm, ck = time_steps(r, k_steps, max(3, a.warmup), dist_on, local)
+            tt = max_over_ranks(tt, dist_on)
+            v, u = workload_value(q, tt / k_steps)
+            rf = roofline(q, pm, peaks, profiled_traffic(name))
+            extras[name] = {"workload": DESCR[name], "value": round(world * v, 3), "unit": u,
+                            "ms_per_step": round(tt / k_steps, 4), "frac_of_peak": rf["frac"],
+                            "roofline": rf, "gpu_launches_per_step": r.launches,
+                            "sm_mhz": ck.get("sm_mhz")}
+            if q.splitkv:
+                extras[name]["num_splits"] = r.ns
+            del q, r
+            torch.cuda.empty_cache()
+
+    # ---- CPU oracle on this host (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and p_cpu is not None:
+        import oracle
+        v, secs, n = time_oracle(p_cpu, a.cpu_seconds)
+        cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+               "kind": "oracle",
+               "sample": f"{n} random (b, h, i) rows of {a.workload}, fp64 C/OpenMP, {secs:.1f} s"}
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) inputs of the workload's shape)",
+        "config": {"workload": f"{a.workload}: {DESCR[a.workload]}",
+                   "global_batch": p.B * world, "seq_len": p.max_seqlen_q,
+                   "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"inputs larger than L2 ({p.hbm_bytes() / 1e6:.0f} MB per step), no flush",
+                   "pct_of_bf16_peak": round(100 * roof["frac"], 2) if roof["bound"] == "tensor" else None},
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": a.steps * run.launches,
+        "clocks": clocks,
+        "kernel_source_sha256": kernel_source_hash(),
+        "workloads": extras,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_reference(a, world):
+    """The CPU oracle as the reference arm: each step computes a bounded
+    random sample of rows of the same workload."""
+    import fa_inputs
+    import oracle
+    name = a.workload
+    p = fa_inputs.make(name) if name not in BIG else None
+    if p is None:
+        print(json.dumps({"impl": "reference", "unavailable":
+                          f"{name}: multi-GB inputs are drawn on the device only"}))
+        return 0
+    # size one step to ~cpu_seconds / steps of CPU work
+    v0, secs0, n0 = time_oracle(p, max(0.5, a.cpu_seconds / max(1, a.steps + a.warmup)))
+    kw = dict(causal=p.causal, softmax_scale=p.softmax_scale, seqused_k=p.seqused_k,
+              rel_bias=p.rel_bias)
+    if p.layout == "varlen":
+        kw.update(cu_seqlens_q=p.cu_seqlens_q, cu_seqlens_k=p.cu_seqlens_k)
+    samples = [oracle_rows_sample(p, n0, seed=s) for s in range(a.warmup + a.steps)]
+    for rows, _ in samples[:a.warmup]:
+        oracle.attention_rows(p.q, p.k, p.v, rows, **kw)
+    flops = 0.0
+    t = time.perf_counter()
+    for rows, f in samples[a.warmup:]:
+        oracle.attention_rows(p.q, p.k, p.v, rows, **kw)
+        flops += f
+    dt = time.perf_counter() - t
+    value = flops / dt / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+            "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+            "ms_per_step": round(1e3 * dt / a.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1) inputs of the workload's shape)",
+            "config": {"workload": f"{name}: {DESCR[name]}", "global_batch": p.B,
+                       "seq_len": p.max_seqlen_q, "parallelism": "CPU oracle"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s",
+                             "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": f"{n0} random rows per step of {name}, fp64 C/OpenMP"},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

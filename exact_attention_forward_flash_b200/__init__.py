@@ -1,0 +1,252 @@
+"""Exact attention forward for B200 (sm_100a): Python binding.
+
+A thin ctypes layer over the C ABI in ``include/fa_b200.h``.  It only
+marshals arguments (device pointers, sizes, the current CUDA stream) and, when
+the caller passes none, allocates the output, LSE and split-KV workspace with
+torch; every step of the computation runs in the library's CUDA kernels.
+
+There is no fallback: if ``libfa_b200.so`` is missing or fails to load, the
+first call raises.  Build it with ``python -m
+exact_attention_forward_flash_b200.build`` (or ``__graft_entry__.build()``).
+
+Entry points (same names as the C ABI):
+
+* ``fa_fwd(q, k, v, ...)`` -- dense [B, S, H, D];
+* ``fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, ...)``
+  -- packed [total, H, D] with cu_seqlens ("mgoin/tml-fa4" contract);
+* ``fa_fwd_splitkv(q, k, v, ...)`` -- dense, keys split and merged by LSE.
+
+Each returns ``(out, lse)``.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfa_b200.so")
+
+FA_OK = 0
+_DTYPES = {torch.bfloat16: 0, torch.float16: 1}
+
+_lib = None
+
+
+class FAError(RuntimeError):
+    """A library call returned a non-OK status."""
+
+    def __init__(self, status: int, name: str, message: str):
+        super().__init__(f"{name}: {message}")
+        self.status = status
+        self.name = name
+
+
+def load_library(path: Optional[str] = None):
+    """Load the shared library (raises if it is absent)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"CUDA library not built: {path} is missing "
+            "(run python -m exact_attention_forward_flash_b200.build)")
+    lib = ctypes.CDLL(path)
+    P, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.fa_fwd.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32,
+                           i32, f32, P, P, i32, P]
+    lib.fa_fwd.restype = i32
+    lib.fa_fwd_varlen.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32,
+                                  i32, i32, i32, i32, i32, i32, f32, P, i32, P]
+    lib.fa_fwd_varlen.restype = i32
+    lib.fa_splitkv_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+    lib.fa_splitkv_workspace_bytes.restype = ctypes.c_size_t
+    lib.fa_splitkv_default_splits.argtypes = [i32, i32, i32, i32, i32, i32, i32]
+    lib.fa_splitkv_default_splits.restype = i32
+    lib.fa_fwd_splitkv.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32,
+                                   i32, i32, i32, f32, P, P, i32, i32, P,
+                                   ctypes.c_size_t, P]
+    lib.fa_fwd_splitkv.restype = i32
+    lib.fa_check_device_error.argtypes = [ctypes.POINTER(i32), i32]
+    lib.fa_check_device_error.restype = i32
+    lib.fa_status_string.argtypes = [i32]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_last_error_message.argtypes = []
+    lib.fa_last_error_message.restype = ctypes.c_char_p
+    lib.fa_version.argtypes = []
+    lib.fa_version.restype = ctypes.c_char_p
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def _check(status: int):
+    if status != FA_OK:
+        lib = load_library()
+        raise FAError(status, lib.fa_status_string(status).decode(),
+                      lib.fa_last_error_message().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        stream = stream.cuda_stream
+    return ctypes.c_void_p(int(stream))
+
+
+def _dtype(q: torch.Tensor) -> int:
+    if q.dtype not in _DTYPES:
+        raise TypeError(f"q must be bf16 or fp16, got {q.dtype}")
+    return _DTYPES[q.dtype]
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("all tensors must be CUDA tensors")
+            if not t.is_contiguous():
+                raise ValueError("all tensors must be contiguous")
+
+
+def _same_dtype(q, *ts):
+    for t in ts:
+        if t is not None and t.dtype != q.dtype:
+            raise TypeError("q, k, v, out and rel_bias must share one dtype")
+
+
+def _int32(t, name):
+    if t is not None and t.dtype != torch.int32:
+        raise TypeError(f"{name} must be int32")
+
+
+def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
+           causal: bool = False, softmax_scale: Optional[float] = None,
+           seqused_k: Optional[torch.Tensor] = None,
+           rel_bias: Optional[torch.Tensor] = None,
+           out: Optional[torch.Tensor] = None,
+           lse: Optional[torch.Tensor] = None,
+           stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Dense forward: q [B,Sq,Hq,D], k/v [B,Sk,Hkv,D] -> (out, lse [B,Hq,Sq])."""
+    lib = load_library()
+    B, Sq, Hq, D = q.shape
+    _, Sk, Hkv, _ = k.shape
+    if k.shape[0] != B or v.shape != k.shape or k.shape[3] != D:
+        raise ValueError("q/k/v shapes disagree")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    _need_cuda(q, k, v, out, lse, seqused_k, rel_bias)
+    _same_dtype(q, k, v, out, rel_bias)
+    _int32(seqused_k, "seqused_k")
+    R = 0 if rel_bias is None else int(rel_bias.shape[-1])
+    _check(lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq,
+                      Sk, Hq, Hkv, D, _dtype(q), int(bool(causal)),
+                      float(softmax_scale or 0.0), _ptr(seqused_k),
+                      _ptr(rel_bias), R, _stream(stream)))
+    return out, lse
+
+
+def fa_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                  cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor,
+                  max_seqlen_q: int, max_seqlen_k: int, *,
+                  seqused_k: Optional[torch.Tensor] = None,
+                  causal: bool = False, softmax_scale: Optional[float] = None,
+                  rel_bias: Optional[torch.Tensor] = None,
+                  out: Optional[torch.Tensor] = None,
+                  lse: Optional[torch.Tensor] = None,
+                  stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Varlen forward: q [total_q,Hq,D], k/v [total_k,Hkv,D] ->
+    (out [total_q,Hq,D], lse [Hq,total_q])."""
+    lib = load_library()
+    total_q, Hq, D = q.shape
+    total_k, Hkv, _ = k.shape
+    B = int(cu_seqlens_q.shape[0]) - 1
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    _need_cuda(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, seqused_k, rel_bias)
+    _same_dtype(q, k, v, out, rel_bias)
+    for t, n in ((cu_seqlens_q, "cu_seqlens_q"), (cu_seqlens_k, "cu_seqlens_k"),
+                 (seqused_k, "seqused_k")):
+        _int32(t, n)
+    R = 0 if rel_bias is None else int(rel_bias.shape[-1])
+    _check(lib.fa_fwd_varlen(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens_q),
+        _ptr(cu_seqlens_k), _ptr(seqused_k), B, int(max_seqlen_q),
+        int(max_seqlen_k), total_q, total_k, Hq, Hkv, D, _dtype(q),
+        int(bool(causal)), float(softmax_scale or 0.0), _ptr(rel_bias), R,
+        _stream(stream)))
+    return out, lse
+
+
+def splitkv_default_splits(B, Sq, Sk, Hq, Hkv, D, num_sms=0) -> int:
+    return int(load_library().fa_splitkv_default_splits(B, Sq, Sk, Hq, Hkv, D, num_sms))
+
+
+def splitkv_workspace_bytes(B, Sq, Hq, D, num_splits) -> int:
+    return int(load_library().fa_splitkv_workspace_bytes(B, Sq, Hq, D, num_splits))
+
+
+def fa_fwd_splitkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
+                   num_splits: int = 0, causal: bool = False,
+                   softmax_scale: Optional[float] = None,
+                   seqused_k: Optional[torch.Tensor] = None,
+                   rel_bias: Optional[torch.Tensor] = None,
+                   out: Optional[torch.Tensor] = None,
+                   lse: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None,
+                   stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Split-KV dense forward (decode); returns (out, lse [B,Hq,Sq])."""
+    lib = load_library()
+    B, Sq, Hq, D = q.shape
+    _, Sk, Hkv, _ = k.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    ns = num_splits
+    if ns <= 0:
+        ns = splitkv_default_splits(B, Sq, Sk, Hq, Hkv, D,
+                                    torch.cuda.get_device_properties(q.device).multi_processor_count)
+    need = splitkv_workspace_bytes(B, Sq, Hq, D, ns)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _need_cuda(q, k, v, out, lse, seqused_k, rel_bias, workspace)
+    _same_dtype(q, k, v, out, rel_bias)
+    _int32(seqused_k, "seqused_k")
+    R = 0 if rel_bias is None else int(rel_bias.shape[-1])
+    _check(lib.fa_fwd_splitkv(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq, Sk, Hq, Hkv,
+        D, _dtype(q), int(bool(causal)), float(softmax_scale or 0.0),
+        _ptr(seqused_k), _ptr(rel_bias), R, int(ns), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out, lse
+
+
+def check_device_error(clear: bool = True) -> int:
+    """Synchronise and return the kernels' watchdog word (0 = no timeout)."""
+    code = ctypes.c_int(0)
+    st = load_library().fa_check_device_error(ctypes.byref(code), int(clear))
+    if st not in (FA_OK, 5):
+        _check(st)
+    return int(code.value)
+
+
+def version() -> str:
+    return load_library().fa_version().decode()
+
+
+def default_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)

@@ -1,0 +1,380 @@
+// fa_api.cu -- the C ABI of the attention forward library (declared in
+// include/fa_b200.h): argument validation, TMA descriptor encoding, kernel
+// selection and launch.  Nothing here allocates device memory or synchronises
+// a stream (fa_check_device_error excepted, by its contract).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "fa_b200.h"
+#include "fa_fwd_kernel.cuh"
+
+namespace {
+
+using namespace fab;
+
+thread_local char g_msg[512] = "";
+
+fa_status fail(fa_status s, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+// ---------------------------------------------------------------------------
+// driver entry point for tensor-map encoding (no link-time libcuda dependency)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D map over a [tokens, heads, D] tensor of 16-bit elements with a box of
+// {64 columns, box_h heads, box_t tokens}, 128-byte swizzle, zero fill.
+fa_status make_map(CUtensorMap *tm, const void *base, int D, int H, long long tokens, int box_h,
+                   int box_t, bool half) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)tokens};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_h, (cuuint32_t)box_t};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(tm, half ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return FA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// per-device state
+// ---------------------------------------------------------------------------
+constexpr int kMaxDev = 64;
+
+int num_sms(int dev) {
+  static int cache[kMaxDev] = {0};
+  if (dev < 0 || dev >= kMaxDev) return 148;
+  if (cache[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      v = 148;
+    cache[dev] = v;
+  }
+  return cache[dev];
+}
+
+// kernel variants
+using Fwd128B = FwdCfg<128, 128, 2, 1, 2, 2, false, false>;
+using Fwd128H = FwdCfg<128, 128, 2, 1, 2, 2, true, false>;
+using Fwd256B = FwdCfg<256, 64, 1, 2, 2, 2, false, false>;
+using Fwd256H = FwdCfg<256, 64, 1, 2, 2, 2, true, false>;
+using Spl128B = FwdCfg<128, 128, 1, 2, 3, 3, false, true>;
+using Spl128H = FwdCfg<128, 128, 1, 2, 3, 3, true, true>;
+using Spl256B = FwdCfg<256, 64, 1, 2, 2, 2, false, true>;
+using Spl256H = FwdCfg<256, 64, 1, 2, 2, 2, true, true>;
+
+template <class C>
+fa_status launch_fwd(FwdParams &p, int dev, cudaStream_t st) {
+  static bool configured[kMaxDev] = {false};
+  if (dev >= 0 && dev < kMaxDev && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(fa_fwd_kernel<C>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess)
+      return fail(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    configured[dev] = true;
+  }
+  const int grid = std::min(p.num_units, num_sms(dev));
+  fa_fwd_kernel<C><<<grid, C::kThreads, C::kSmemBytes, st>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
+  return FA_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr unsigned long long kTimeoutNs = 4000000000ull;  // 4 s per wait
+
+struct Common {
+  const void *q, *k, *v;
+  void *out;
+  float *lse;
+  const int *cu_q, *cu_k, *seqused_k;
+  const void *rel_bias;
+  int R, B, Sq, Sk, Hq, Hkv, D, total_q, total_k, max_q;
+  fa_dtype dt;
+  int causal;
+  float scale;
+  bool varlen;
+};
+
+fa_status validate(const Common &c) {
+  if (c.dt != FA_BF16 && c.dt != FA_FP16) return fail(FA_ERR_INVALID, "dtype must be bf16 or fp16");
+  if (c.B < 0 || c.Hq <= 0 || c.Hkv <= 0 || c.D <= 0)
+    return fail(FA_ERR_INVALID, "B must be >= 0 and Hq, Hkv, D > 0");
+  if (c.Hq % c.Hkv != 0) return fail(FA_ERR_INVALID, "Hq (%d) must be a multiple of Hkv (%d)", c.Hq, c.Hkv);
+  if (c.D != 128 && c.D != 256)
+    return fail(FA_ERR_UNSUPPORTED, "head_dim %d not served (128 or 256)", c.D);
+  if (!c.varlen && (c.Sq < 0 || c.Sk < 0)) return fail(FA_ERR_INVALID, "Sq, Sk must be >= 0");
+  if (c.varlen && (c.total_q < 0 || c.total_k < 0 || c.max_q < 0))
+    return fail(FA_ERR_INVALID, "total_q, total_k, max_seqlen_q must be >= 0");
+  if (c.rel_bias != nullptr) {
+    if (c.R <= 0 || c.R % 128 != 0)
+      return fail(FA_ERR_INVALID, "rel_extent (%d) must be a positive multiple of 128", c.R);
+    if (!aligned16(c.rel_bias)) return fail(FA_ERR_INVALID, "rel_bias must be 16-byte aligned");
+  }
+  if (!std::isfinite(c.scale)) return fail(FA_ERR_INVALID, "softmax_scale must be finite");
+  const long long tq = c.varlen ? c.total_q : (long long)c.B * c.Sq;
+  const long long tk = c.varlen ? c.total_k : (long long)c.B * c.Sk;
+  if (tq > 0x7fffffffLL || tk > 0x7fffffffLL || tq * c.Hq > (1LL << 40))
+    return fail(FA_ERR_UNSUPPORTED, "problem too large for 32-bit token indices");
+  if (tq > 0) {
+    if (!c.q || !c.out) return fail(FA_ERR_INVALID, "q and out must not be NULL");
+    if (!aligned16(c.q) || !aligned16(c.out)) return fail(FA_ERR_INVALID, "q/out must be 16-byte aligned");
+    if (tk > 0) {
+      if (!c.k || !c.v) return fail(FA_ERR_INVALID, "k and v must not be NULL");
+      if (!aligned16(c.k) || !aligned16(c.v)) return fail(FA_ERR_INVALID, "k/v must be 16-byte aligned");
+    }
+  }
+  if (c.varlen && c.B > 0 && (!c.cu_q || !c.cu_k))
+    return fail(FA_ERR_INVALID, "cu_seqlens_q and cu_seqlens_k must not be NULL");
+  return FA_OK;
+}
+
+// Query heads packed per tile: all heads of a K/V group when that divides 128.
+int pack_factor(int G) { return (G >= 1 && G <= 128 && 128 % G == 0) ? G : 1; }
+
+fa_status fill_params(const Common &c, FwdParams &p, int nq, int bn, int num_splits,
+                      int split_keys) {
+  std::memset(&p, 0, sizeof(p));
+  const bool half = c.dt == FA_FP16;
+  const int G = c.Hq / c.Hkv;
+  const int P = pack_factor(G);
+  const long long tq = c.varlen ? c.total_q : (long long)c.B * c.Sq;
+  const long long tk = c.varlen ? c.total_k : (long long)c.B * c.Sk;
+  fa_status s;
+  if ((s = make_map(&p.tm_q, c.q, c.D, c.Hq, tq, P, kBM / P, half)) != FA_OK) return s;
+  // With no keys at all every unit is empty and K/V are never read; the maps
+  // then describe one token of q (which holds at least Hkv * D elements).
+  const void *kb = tk > 0 ? c.k : c.q;
+  const void *vb = tk > 0 ? c.v : c.q;
+  const long long tkm = tk > 0 ? tk : 1;
+  if ((s = make_map(&p.tm_k, kb, c.D, c.Hkv, tkm, 1, bn, half)) != FA_OK) return s;
+  if ((s = make_map(&p.tm_v, vb, c.D, c.Hkv, tkm, 1, bn, half)) != FA_OK) return s;
+  p.out = c.out;
+  p.lse = c.lse;
+  p.cu_q = c.varlen ? c.cu_q : nullptr;
+  p.cu_k = c.varlen ? c.cu_k : nullptr;
+  p.seqused_k = c.seqused_k;
+  p.rel_bias = static_cast<const uint16_t *>(c.rel_bias);
+  p.R = c.rel_bias ? c.R : 0;
+  p.B = c.B;
+  p.Sq = c.Sq;
+  p.Sk = c.Sk;
+  p.Hq = c.Hq;
+  p.Hkv = c.Hkv;
+  p.G = G;
+  p.P = P;
+  p.n_groups = c.Hq / P;
+  p.total_q = (int)tq;
+  const int max_q = c.varlen ? c.max_q : c.Sq;
+  const long long rows = (long long)max_q * P;
+  p.n_mblk = (int)std::max<long long>(1, (rows + (long long)nq * kBM - 1) / ((long long)nq * kBM));
+  p.num_splits = num_splits;
+  p.split_keys = split_keys;
+  p.causal = c.causal ? 1 : 0;
+  p.lse_dense = c.varlen ? 0 : 1;
+  const long long units = (long long)c.B * p.n_groups * p.n_mblk * num_splits;
+  if (units > 0x7fffffffLL) return fail(FA_ERR_UNSUPPORTED, "too many work units");
+  p.num_units = (int)units;
+  const float scale = c.scale > 0.f ? c.scale : 1.0f / std::sqrt((float)c.D);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.inv_scale = 1.0f / scale;
+  p.thr_raw = 8.0f / p.scale_log2;
+  p.timeout_ns = kTimeoutNs;
+  return FA_OK;
+}
+
+fa_status run_fwd(const Common &c, cudaStream_t st) {
+  fa_status s = validate(c);
+  if (s != FA_OK) return s;
+  const long long tq = c.varlen ? c.total_q : (long long)c.B * c.Sq;
+  if (tq == 0 || c.B == 0) return FA_OK;  // nothing to compute
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(FA_ERR_CUDA, "cudaGetDevice failed");
+  FwdParams p;
+  if ((s = fill_params(c, p, c.D == 128 ? 2 : 1, c.D == 128 ? 128 : 64, 1, 0x7fffffff)) != FA_OK)
+    return s;
+  if (p.num_units == 0) return FA_OK;
+  const bool half = c.dt == FA_FP16;
+  if (c.D == 128) return half ? launch_fwd<Fwd128H>(p, dev, st) : launch_fwd<Fwd128B>(p, dev, st);
+  return half ? launch_fwd<Fwd256H>(p, dev, st) : launch_fwd<Fwd256B>(p, dev, st);
+}
+
+template <int D, bool HALF>
+fa_status launch_combine(const float *o_part, const float *lse_part, int ns, long long rows,
+                         void *out, float *lse, int Hq, int Sq, int total_q, int lse_dense,
+                         cudaStream_t st) {
+  const int warps = 8;
+  const long long blocks = (rows + warps - 1) / warps;
+  if (blocks > 0x7fffffffLL) return fail(FA_ERR_UNSUPPORTED, "too many rows");
+  fa_combine_kernel<D, HALF><<<(unsigned)blocks, warps * 32, 0, st>>>(
+      o_part, lse_part, ns, rows, out, lse, Hq, Sq, total_q, lse_dense);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
+  return FA_OK;
+}
+
+int splitkv_bn(int D) { return D == 128 ? 128 : 64; }
+
+}  // namespace
+
+extern "C" {
+
+const char *fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID: return "FA_ERR_INVALID";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT";
+  }
+  return "FA_ERR_UNKNOWN";
+}
+
+const char *fa_last_error_message(void) { return g_msg; }
+
+const char *fa_version(void) { return "fa_b200 0.1 (sm_100a)"; }
+
+fa_status fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse, int B,
+                 int Sq, int Sk, int Hq, int Hkv, int D, fa_dtype dt, int causal,
+                 float softmax_scale, const int *seqused_k, const void *rel_bias, int rel_extent,
+                 void *stream) {
+  g_msg[0] = 0;
+  Common c{q, k, v, out, lse, nullptr, nullptr, seqused_k, rel_bias, rel_extent, B, Sq, Sk,
+           Hq, Hkv, D, 0, 0, 0, dt, causal, softmax_scale, false};
+  return run_fwd(c, static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_fwd_varlen(const void *q, const void *k, const void *v, void *out, float *lse,
+                        const int *cu_seqlens_q, const int *cu_seqlens_k, const int *seqused_k,
+                        int B, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                        int Hq, int Hkv, int D, fa_dtype dt, int causal, float softmax_scale,
+                        const void *rel_bias, int rel_extent, void *stream) {
+  g_msg[0] = 0;
+  (void)max_seqlen_k;
+  Common c{q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, seqused_k, rel_bias, rel_extent, B,
+           0, 0, Hq, Hkv, D, total_q, total_k, max_seqlen_q, dt, causal, softmax_scale, true};
+  return run_fwd(c, static_cast<cudaStream_t>(stream));
+}
+
+size_t fa_splitkv_workspace_bytes(int B, int Sq, int Hq, int D, int num_splits) {
+  if (B <= 0 || Sq <= 0 || Hq <= 0 || D <= 0 || num_splits <= 0) return 0;
+  const size_t rows = (size_t)B * Sq * Hq;
+  size_t bytes = (size_t)num_splits * rows * (size_t)(D + 1) * sizeof(float);
+  return (bytes + 255) & ~(size_t)255;
+}
+
+int fa_splitkv_default_splits(int B, int Sq, int Sk, int Hq, int Hkv, int D, int n_sms) {
+  if (B <= 0 || Sq <= 0 || Sk <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv) return 1;
+  if (n_sms <= 0) n_sms = 148;
+  const int bn = splitkv_bn(D);
+  const int P = pack_factor(Hq / Hkv);
+  const long long mblk = ((long long)Sq * P + kBM - 1) / kBM;
+  const long long base = (long long)B * (Hq / P) * mblk;  // units without splitting
+  const long long max_by_len = std::max<long long>(1, ((long long)Sk + 8 * bn - 1) / (8 * bn));
+  if (base >= 4LL * n_sms) return 1;
+  // enough units for about 16 per SM, in whole waves where possible
+  long long ns = (16LL * n_sms + base - 1) / base;
+  ns = std::min(ns, max_by_len);
+  ns = std::min<long long>(ns, 256);
+  return (int)std::max<long long>(1, ns);
+}
+
+fa_status fa_fwd_splitkv(const void *q, const void *k, const void *v, void *out, float *lse,
+                         int B, int Sq, int Sk, int Hq, int Hkv, int D, fa_dtype dt, int causal,
+                         float softmax_scale, const int *seqused_k, const void *rel_bias,
+                         int rel_extent, int num_splits, void *workspace, size_t workspace_bytes,
+                         void *stream) {
+  g_msg[0] = 0;
+  Common c{q, k, v, out, lse, nullptr, nullptr, seqused_k, rel_bias, rel_extent, B, Sq, Sk,
+           Hq, Hkv, D, 0, 0, 0, dt, causal, softmax_scale, false};
+  fa_status s = validate(c);
+  if (s != FA_OK) return s;
+  if (num_splits < 0) return fail(FA_ERR_INVALID, "num_splits must be >= 0");
+  if ((long long)B * Sq == 0) return FA_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(FA_ERR_CUDA, "cudaGetDevice failed");
+  if (Sk == 0) return run_fwd(c, st);  // nothing to split
+  const int bn = splitkv_bn(D);
+  int ns = num_splits > 0 ? num_splits : fa_splitkv_default_splits(B, Sq, Sk, Hq, Hkv, D, num_sms(dev));
+  long long tiles = ((long long)Sk + bn - 1) / bn;
+  if (ns > tiles) ns = (int)tiles;
+  const int split_keys = (int)(((tiles + ns - 1) / ns) * bn);
+  ns = (int)(((long long)Sk + split_keys - 1) / split_keys);
+  const size_t need = fa_splitkv_workspace_bytes(B, Sq, Hq, D, ns);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(FA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+  if (!aligned16(workspace)) return fail(FA_ERR_INVALID, "workspace must be 16-byte aligned");
+  FwdParams p;
+  if ((s = fill_params(c, p, 1, bn, ns, split_keys)) != FA_OK) return s;
+  const long long rows = (long long)B * Sq * Hq;
+  p.o_part = static_cast<float *>(workspace);
+  p.lse_part = p.o_part + (size_t)ns * rows * D;
+  const bool half = dt == FA_FP16;
+  if (D == 128)
+    s = half ? launch_fwd<Spl128H>(p, dev, st) : launch_fwd<Spl128B>(p, dev, st);
+  else
+    s = half ? launch_fwd<Spl256H>(p, dev, st) : launch_fwd<Spl256B>(p, dev, st);
+  if (s != FA_OK) return s;
+  if (D == 128)
+    return half ? launch_combine<128, true>(p.o_part, p.lse_part, ns, rows, out, lse, Hq, Sq,
+                                            B * Sq, 1, st)
+                : launch_combine<128, false>(p.o_part, p.lse_part, ns, rows, out, lse, Hq, Sq,
+                                             B * Sq, 1, st);
+  return half ? launch_combine<256, true>(p.o_part, p.lse_part, ns, rows, out, lse, Hq, Sq,
+                                          B * Sq, 1, st)
+              : launch_combine<256, false>(p.o_part, p.lse_part, ns, rows, out, lse, Hq, Sq,
+                                           B * Sq, 1, st);
+}
+
+fa_status fa_check_device_error(int *code, int clear) {
+  unsigned v = 0;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "cudaDeviceSynchronize: %s", cudaGetErrorString(e));
+  e = cudaMemcpyFromSymbol(&v, fab::g_fa_error, sizeof(v));
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "reading the error word: %s", cudaGetErrorString(e));
+  if (code) *code = (int)v;
+  if (clear && v) {
+    unsigned z = 0;
+    e = cudaMemcpyToSymbol(fab::g_fa_error, &z, sizeof(z));
+    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "clearing the error word: %s", cudaGetErrorString(e));
+  }
+  return v ? FA_ERR_DEVICE_TIMEOUT : FA_OK;
+}
+
+}  // extern "C"

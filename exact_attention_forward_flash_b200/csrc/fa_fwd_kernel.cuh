@@ -1,0 +1,670 @@
+// fa_fwd_kernel.cuh -- the attention forward kernel for sm_100a.
+//
+// Computes O = softmax(scale * Q K^T + bias + mask) V and its log-sum-exp
+// tile by tile with an online softmax, so the score matrix never leaves the
+// chip.  The operation, the distance rule and the layouts follow the pages:
+// "mgoin/tml-fa4" (argument contract: varlen layout, cu_seqlens, the distance
+// d = i + (k_len - q_len) - j, rel_bias added for 0 <= d < rel_extent, causal
+// meaning of d) and "flashrt/fa4-cute-runtime" ((out, lse) results,
+// seqused_k, packed GQA heads).  The online softmax (running max, normaliser,
+// P.V accumulation) is the loop that "ATFlash-Kernel-FA4" (What the window
+// does) describes.
+//
+// Structure of one CTA (persistent; it walks work units u = blockIdx.x,
+// blockIdx.x + gridDim.x, ...):
+//
+//   warp 0      TMA producer: Q tiles once per unit, then K and V tiles of
+//               BN keys through separate KST-/VST-stage shared-memory rings.
+//   warp 1      MMA issuer (one thread): S = Q K^T (SS form, both operands
+//               K-major in 128B-swizzled shared memory) into tensor memory,
+//               and O += P V (TS form: P read from tensor memory where it
+//               overwrites S, V MN-major in shared memory).  Also owns the
+//               tensor-memory allocation.
+//   warps 2,3   idle.
+//   warps 4..   one 128-thread softmax warpgroup per Q tile; thread r owns
+//               tile row r (= TMEM lane r).  Per KV tile it loads its score
+//               row from tensor memory, adds the relative bias, applies the
+//               masks, updates the running max, rescales O in tensor memory
+//               only when the max has grown by more than 2^8 (conditional
+//               rescaling), writes P = exp2(.) back as 16-bit pairs, and
+//               after the last tile normalises O and writes O and the LSE.
+//
+// A Q tile holds 128 packed rows: P consecutive query heads that share one
+// K/V head (P = Hq/Hkv when that divides 128, else 1) at 128/P consecutive
+// positions, loaded with one 3-D TMA box {64, P, 128/P} per 64 columns.
+//
+// Every wait is bounded (see mbar_wait); a role that gives up records the
+// timeout in g_fa_error, drains what it has in flight, and leaves its loops.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "sm100_ptx.cuh"
+
+namespace fab {
+
+__device__ unsigned g_fa_error;  // watchdog word, read by fa_check_device_error
+
+constexpr int kBM = 128;  // rows per Q tile = TMEM lanes
+
+struct FwdParams {
+  CUtensorMap tm_q, tm_k, tm_v;  // 3-D maps over [tokens, heads, D]
+  void *out;                     // final output (input dtype), packed [tok, Hq, D]
+  float *lse;                    // final LSE, or nullptr
+  float *o_part;                 // split partials [splits][tok*Hq][D] fp32
+  float *lse_part;               // split partial LSE [splits][tok*Hq]
+  const int *cu_q, *cu_k;        // varlen offsets, nullptr when dense
+  const int *seqused_k;          // nullptr or [B]
+  const uint16_t *rel_bias;      // nullptr or [tok, Hq, R]
+  int R;
+  int B, Sq, Sk, Hq, Hkv, G, P, n_groups;
+  int total_q;
+  int n_mblk;        // CTA tiles per (batch, head group, split)
+  int num_splits;
+  int split_keys;    // keys per split (multiple of BN); >= any k_len when 1 split
+  int causal;
+  int lse_dense;     // 1: lse [B, Hq, Sq]; 0: lse [Hq, total_q]
+  int num_units;
+  float scale_log2;  // softmax_scale * log2(e)
+  float inv_scale;   // 1 / softmax_scale (bias is folded into raw-score units)
+  float thr_raw;     // rescale threshold 8 (log2 units) in raw-score units
+  unsigned long long timeout_ns;
+};
+
+// One work unit: NQ Q tiles of one (batch, head group) and one key split.
+struct Unit {
+  int b, hq0, hk, split;
+  int q_start, q_len, k_start, k_len, delta;
+  int row0;          // first packed row of tile 0 within the sequence
+  int kv_lo, kv_hi;  // key range handled by this unit
+  int nb;            // KV tiles
+  unsigned active;   // bit t: tile t holds at least one valid row
+};
+
+template <int NQ, int BN>
+__device__ __forceinline__ bool decode_unit(const FwdParams &p, int u, Unit &U) {
+  int mblk_rev = u % p.n_mblk;
+  int rest = u / p.n_mblk;
+  U.split = rest % p.num_splits;
+  rest /= p.num_splits;
+  const int grp = rest % p.n_groups;
+  U.b = rest / p.n_groups;
+  const int mblk = p.n_mblk - 1 - mblk_rev;  // heaviest causal tiles first
+  U.hq0 = grp * p.P;
+  U.hk = U.hq0 / p.G;
+  if (p.cu_q != nullptr) {
+    U.q_start = __ldg(p.cu_q + U.b);
+    U.q_len = __ldg(p.cu_q + U.b + 1) - U.q_start;
+    U.k_start = __ldg(p.cu_k + U.b);
+    U.k_len = __ldg(p.cu_k + U.b + 1) - U.k_start;
+  } else {
+    U.q_start = U.b * p.Sq;
+    U.q_len = p.Sq;
+    U.k_start = U.b * p.Sk;
+    U.k_len = p.Sk;
+  }
+  if (p.seqused_k != nullptr) U.k_len = min(max(__ldg(p.seqused_k + U.b), 0), U.k_len);
+  U.row0 = mblk * NQ * kBM;
+  if (U.row0 / p.P >= U.q_len) return false;  // no row of this unit exists
+  U.active = 0;
+#pragma unroll
+  for (int t = 0; t < NQ; ++t)
+    if ((U.row0 + t * kBM) / p.P < U.q_len) U.active |= 1u << t;
+  U.delta = U.k_len - U.q_len;
+  const long long lo = (long long)U.split * p.split_keys;
+  long long hi = min((long long)U.k_len, lo + p.split_keys);
+  if (p.causal) {
+    const int i_max = min(U.q_len - 1, (U.row0 + NQ * kBM - 1) / p.P);
+    hi = min(hi, (long long)i_max + U.delta + 1);
+  }
+  U.kv_lo = (int)lo;
+  U.kv_hi = (int)max(hi, lo);
+  U.nb = (U.kv_hi - U.kv_lo + BN - 1) / BN;
+  return true;
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout: start
+// address, leading and stride byte offsets in 16-byte units, version 1,
+// layout type 2 = SWIZZLE_128B).
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;
+  d |= 2ull << 61;
+  return d;
+}
+
+// Instruction descriptor of tcgen05.mma kind::f16 with an fp32 accumulator.
+template <bool kHalf>
+__host__ __device__ constexpr uint32_t instr_desc(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4)                                  // D format: f32
+         | ((kHalf ? 0u : 1u) << 7)                 // A: f16 / bf16
+         | ((kHalf ? 0u : 1u) << 10)                // B: f16 / bf16
+         | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16)
+         | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+template <int D_, int BN_, int NQ_, int NS_, int KST_, int VST_, bool HALF_, bool PARTIAL_>
+struct FwdCfg {
+  static constexpr int D = D_, BN = BN_, NQ = NQ_, NS = NS_, KST = KST_, VST = VST_;
+  static constexpr bool HALF = HALF_, PARTIAL = PARTIAL_;
+  static constexpr int kChunks = D / 64;          // 128-byte column chunks of a row
+  static constexpr int kQTile = kBM * D * 2;      // bytes
+  static constexpr int kKVTile = BN * D * 2;
+  static constexpr int kQChunk = kBM * 128;       // bytes of one 64-column chunk
+  static constexpr int kKVChunk = BN * 128;
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQOff + NQ * kQTile;
+  static constexpr int kVOff = kKOff + KST * kKVTile;
+  static constexpr int kBarOff = kVOff + VST * kKVTile;
+  // barrier indices
+  static constexpr int bQFull = 0, bQEmpty = NQ, bKFull = 2 * NQ, bKEmpty = bKFull + KST,
+                       bVFull = bKEmpty + KST, bVEmpty = bVFull + VST, bSFull = bVEmpty + VST,
+                       bPFull = bSFull + NQ * NS, bOFull = bPFull + NQ * NS,
+                       bOEmpty = bOFull + NQ * NS, bDrain = bOEmpty + NQ, kNumBars = bDrain + 1;
+  static constexpr int kSlotOff = kBarOff + kNumBars * 8;
+  static constexpr int kSmemBytes = kSlotOff + 16 + 1024;  // + alignment slack
+  static constexpr int kThreads = 128 * (1 + NQ);
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr int kOColBase = NQ * NS * BN;
+  static_assert(kOColBase + NQ * D <= 512, "tensor memory budget");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(D % 64 == 0 && BN % 32 == 0 && (BN == 64 || BN == 128), "tile shape");
+  __host__ __device__ static constexpr int s_col(int t, int b) { return (t * NS + b) * BN; }
+  __host__ __device__ static constexpr int o_col(int t) { return kOColBase + t * D; }
+};
+
+// ---------------------------------------------------------------------------
+// producer
+// ---------------------------------------------------------------------------
+template <class C>
+__device__ __forceinline__ void role_producer(const FwdParams &p, uint32_t sb) {
+  auto bar = [&](int i) { return sb + C::kBarOff + 8u * i; };
+  uint32_t q_cnt[C::NQ];
+#pragma unroll
+  for (int t = 0; t < C::NQ; ++t) q_cnt[t] = 0;
+  uint32_t k_cnt = 0, v_cnt = 0;
+  bool ok = true;
+  for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+    Unit U;
+    if (!decode_unit<C::NQ, C::BN>(p, u, U) || U.nb == 0) continue;
+#pragma unroll
+    for (int t = 0; t < C::NQ; ++t) {
+      if (!(U.active >> t & 1u)) continue;
+      ok = mbar_wait(bar(C::bQEmpty + t), (q_cnt[t] & 1u) ^ 1u, &g_fa_error, p.timeout_ns);
+      if (!ok) break;
+      mbar_arrive_expect_tx(bar(C::bQFull + t), C::kQTile);
+      const int tok = U.q_start + (U.row0 + t * kBM) / p.P;
+#pragma unroll
+      for (int c = 0; c < C::kChunks; ++c)
+        tma_load_3d(sb + C::kQOff + t * C::kQTile + c * C::kQChunk, &p.tm_q, c * 64, U.hq0, tok,
+                    bar(C::bQFull + t));
+      ++q_cnt[t];
+    }
+    for (int n = 0; n < U.nb && ok; ++n) {
+      const int tok = U.k_start + U.kv_lo + n * C::BN;
+      {
+        const uint32_t s = k_cnt % C::KST;
+        ok = mbar_wait(bar(C::bKEmpty + s), ((k_cnt / C::KST) & 1u) ^ 1u, &g_fa_error,
+                       p.timeout_ns);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(C::bKFull + s), C::kKVTile);
+#pragma unroll
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_3d(sb + C::kKOff + s * C::kKVTile + c * C::kKVChunk, &p.tm_k, c * 64, U.hk,
+                      tok, bar(C::bKFull + s));
+        ++k_cnt;
+      }
+      {
+        const uint32_t s = v_cnt % C::VST;
+        ok = mbar_wait(bar(C::bVEmpty + s), ((v_cnt / C::VST) & 1u) ^ 1u, &g_fa_error,
+                       p.timeout_ns);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(C::bVFull + s), C::kKVTile);
+#pragma unroll
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_3d(sb + C::kVOff + s * C::kKVTile + c * C::kKVChunk, &p.tm_v, c * 64, U.hk,
+                      tok, bar(C::bVFull + s));
+        ++v_cnt;
+      }
+    }
+  }
+  if (!ok) {
+    // Drain: let every copy this thread issued land before the CTA leaves.
+    const uint64_t drain_ns = 200000000ull;
+    for (uint32_t i = (k_cnt > C::KST ? k_cnt - C::KST : 0); i < k_cnt; ++i)
+      mbar_wait_drain(bar(C::bKFull + i % C::KST), (i / C::KST) & 1u, drain_ns);
+    for (uint32_t i = (v_cnt > C::VST ? v_cnt - C::VST : 0); i < v_cnt; ++i)
+      mbar_wait_drain(bar(C::bVFull + i % C::VST), (i / C::VST) & 1u, drain_ns);
+#pragma unroll
+    for (int t = 0; t < C::NQ; ++t)
+      if (q_cnt[t]) mbar_wait_drain(bar(C::bQFull + t), (q_cnt[t] - 1) & 1u, drain_ns);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// MMA issuer (one thread)
+// ---------------------------------------------------------------------------
+template <class C>
+__device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32_t tmem) {
+  auto bar = [&](int i) { return sb + C::kBarOff + 8u * i; };
+  constexpr uint32_t idesc_s = instr_desc<C::HALF>(kBM, C::BN, false, false);
+  constexpr uint32_t idesc_pv = instr_desc<C::HALF>(kBM, C::D, false, true);
+  uint32_t q_cnt[C::NQ], s_cnt[C::NQ], u_cnt[C::NQ];
+#pragma unroll
+  for (int t = 0; t < C::NQ; ++t) q_cnt[t] = s_cnt[t] = u_cnt[t] = 0;
+  uint32_t k_cnt = 0, v_cnt = 0;
+  bool ok = true;
+
+  // S_t(n) = Q_t K_n^T into the S buffer of global index g
+  auto issue_s = [&](int t, uint32_t g, uint32_t kstage) {
+    const uint32_t qa = sb + C::kQOff + t * C::kQTile;
+    const uint32_t ka = sb + C::kKOff + kstage * C::kKVTile;
+    const uint32_t d_tmem = tmem + C::s_col(t, g % C::NS);
+#pragma unroll
+    for (int kk = 0; kk < C::D / 16; ++kk) {
+      const uint32_t off = (kk % 4) * 32;  // 16 elements = 32 bytes inside the swizzle atom
+      const uint64_t a = smem_desc_sw128(qa + (kk / 4) * C::kQChunk + off, 16, 1024);
+      const uint64_t b = smem_desc_sw128(ka + (kk / 4) * C::kKVChunk + off, 16, 1024);
+      tc_mma_ss(d_tmem, a, b, idesc_s, kk > 0 ? 1u : 0u);
+    }
+    tc_commit(bar(C::bSFull + t * C::NS + g % C::NS));
+  };
+  // O_t += P_t(g) V (P in the S buffer of g, as 16-bit pairs)
+  auto issue_pv = [&](int t, uint32_t g, uint32_t vstage, bool first) {
+    const uint32_t va = sb + C::kVOff + vstage * C::kKVTile;
+    const uint32_t p_tmem = tmem + C::s_col(t, g % C::NS);
+    const uint32_t d_tmem = tmem + C::o_col(t);
+#pragma unroll
+    for (int kk = 0; kk < C::BN / 16; ++kk) {
+      // 16 keys = two 8-row groups (SBO 1024 B); 64-column chunks LBO apart
+      const uint64_t b = smem_desc_sw128(va + kk * 16 * 128, C::kKVChunk, 1024);
+      tc_mma_ts(d_tmem, p_tmem + kk * 8, b, idesc_pv, (first && kk == 0) ? 0u : 1u);
+    }
+    tc_commit(bar(C::bOFull + t * C::NS + g % C::NS));
+  };
+
+  for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+    Unit U;
+    if (!decode_unit<C::NQ, C::BN>(p, u, U) || U.nb == 0) continue;
+    const int nb = U.nb;
+    const int last_t = (U.active >> 1 & 1u) && C::NQ > 1 ? 1 : 0;
+    uint32_t sbase[C::NQ];
+#pragma unroll
+    for (int t = 0; t < C::NQ; ++t) {
+      sbase[t] = s_cnt[t];
+      if (!(U.active >> t & 1u)) continue;
+      ok = ok && mbar_wait(bar(C::bQFull + t), q_cnt[t] & 1u, &g_fa_error, p.timeout_ns);
+      ++q_cnt[t];
+    }
+    if (!ok) break;
+    tc_fence_after();
+    const uint32_t kb = k_cnt, vb = v_cnt;
+
+    // prologue: S(0) for every active tile
+    ok = mbar_wait(bar(C::bKFull + kb % C::KST), (kb / C::KST) & 1u, &g_fa_error, p.timeout_ns);
+    if (!ok) break;
+    tc_fence_after();
+#pragma unroll
+    for (int t = 0; t < C::NQ; ++t) {
+      if (!(U.active >> t & 1u)) continue;
+      issue_s(t, sbase[t], kb % C::KST);
+      if (nb == 1) tc_commit(bar(C::bQEmpty + t));
+    }
+    tc_commit(bar(C::bKEmpty + kb % C::KST));
+
+    for (int n = 0; n < nb && ok; ++n) {
+      const uint32_t kn = kb + n + 1;  // K tile of block n+1
+      if (C::NS == 2 && n + 1 < nb) {
+        ok = mbar_wait(bar(C::bKFull + kn % C::KST), (kn / C::KST) & 1u, &g_fa_error,
+                       p.timeout_ns);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int t = 0; t < C::NQ; ++t) {
+          if (!(U.active >> t & 1u)) continue;
+          issue_s(t, sbase[t] + n + 1, kn % C::KST);
+          if (n + 1 == nb - 1) tc_commit(bar(C::bQEmpty + t));
+        }
+        tc_commit(bar(C::bKEmpty + kn % C::KST));
+      }
+      const uint32_t vn = vb + n;
+      ok = mbar_wait(bar(C::bVFull + vn % C::VST), (vn / C::VST) & 1u, &g_fa_error,
+                     p.timeout_ns);
+      if (!ok) break;
+#pragma unroll
+      for (int t = 0; t < C::NQ; ++t) {
+        if (!(U.active >> t & 1u)) continue;
+        const uint32_t g = sbase[t] + n;
+        if (n == 0) {
+          ok = mbar_wait(bar(C::bOEmpty + t), (u_cnt[t] & 1u) ^ 1u, &g_fa_error, p.timeout_ns);
+          if (!ok) break;
+        }
+        ok = mbar_wait(bar(C::bPFull + t * C::NS + g % C::NS), (g / C::NS) & 1u, &g_fa_error,
+                       p.timeout_ns);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(t, g, vn % C::VST, n == 0);
+        if (t == last_t) tc_commit(bar(C::bVEmpty + vn % C::VST));
+        if (C::NS == 1 && n + 1 < nb) {
+          if (t == 0) {
+            ok = mbar_wait(bar(C::bKFull + kn % C::KST), (kn / C::KST) & 1u, &g_fa_error,
+                           p.timeout_ns);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          issue_s(t, g + 1, kn % C::KST);
+          if (n + 1 == nb - 1) tc_commit(bar(C::bQEmpty + t));
+          if (t == last_t) tc_commit(bar(C::bKEmpty + kn % C::KST));
+        }
+      }
+    }
+    k_cnt += nb;
+    v_cnt += nb;
+#pragma unroll
+    for (int t = 0; t < C::NQ; ++t) {
+      if (!(U.active >> t & 1u)) continue;
+      s_cnt[t] += nb;
+      ++u_cnt[t];
+    }
+  }
+  // Wait for every MMA this thread issued before tensor memory is released.
+  tc_commit(bar(C::bDrain));
+  mbar_wait_drain(bar(C::bDrain), 0, ok ? p.timeout_ns : 200000000ull);
+}
+
+// ---------------------------------------------------------------------------
+// softmax / correction / epilogue warpgroup (one per Q tile)
+// ---------------------------------------------------------------------------
+template <class C>
+__device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, uint32_t tmem,
+                                             int t) {
+  auto bar = [&](int i) { return sb + C::kBarOff + 8u * i; };
+  constexpr int BN = C::BN, D = C::D, NS = C::NS;
+  const int tid = static_cast<int>(threadIdx.x) - 128 * (t + 1);  // tile row == TMEM lane
+  const uint32_t lane_addr = static_cast<uint32_t>(tid & ~31) << 16;
+  const float sl2 = p.scale_log2;
+  uint32_t s_cnt = 0;
+  bool ok = true;
+
+  for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+    Unit U;
+    if (!decode_unit<C::NQ, BN>(p, u, U) || !(U.active >> t & 1u)) continue;
+    const int row = U.row0 + t * kBM + tid;
+    const int i = row / p.P;
+    const int h = U.hq0 + row % p.P;
+    const bool valid = i < U.q_len;
+    const bool warp_on = __any_sync(0xffffffffu, valid);
+    const int lim = p.causal ? min(U.kv_hi, i + U.delta + 1) : U.kv_hi;  // keys j < lim
+    const uint16_t *brow = nullptr;
+    if (p.rel_bias != nullptr && valid)
+      brow = p.rel_bias + ((size_t)(U.q_start + i) * p.Hq + h) * p.R;
+
+    float m_ref = -INFINITY, l = 0.f;
+    for (int n = 0; n < U.nb; ++n) {
+      const uint32_t g = s_cnt + n;
+      const uint32_t buf = g % NS;
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(bar(C::bSFull + t * NS + buf), (g / NS) & 1u, &g_fa_error,
+                                p.timeout_ns));
+      if (!ok) break;
+      tc_fence_after();
+      if (warp_on) {
+        const uint32_t s_addr = tmem + lane_addr + C::s_col(t, buf);
+        float s[BN];
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(s_addr + 32 * c, r);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(r[e]);
+        }
+        tmem_wait_ld();
+        const int j0 = U.kv_lo + n * BN;
+        // relative bias: column c sits at distance d = base - c
+        if (brow != nullptr) {
+          const int base = i + U.delta - j0;
+          if (base >= 0 && base - (BN - 1) < p.R) {
+#pragma unroll
+            for (int c = 0; c < BN; ++c) {
+              const int d = base - c;
+              if (d >= 0 && d < p.R) s[c] += load_elem<C::HALF>(brow + d) * p.inv_scale;
+            }
+          }
+        }
+        // masks: keys at or past `lim` (end of keys / causal diagonal)
+        const int lim_c = lim - j0;
+        if (lim_c < BN) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (c >= lim_c) s[c] = -INFINITY;
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+        const float m_new = fmaxf(m_ref, mx);
+        if (n == 0) {
+          m_ref = m_new;
+        } else {
+          const bool need = (m_new - m_ref) > p.thr_raw;
+          if (__any_sync(0xffffffffu, need)) {
+            if (NS == 2) {  // the previous P.V must have landed in O
+              const uint32_t gp = g - 1;
+              ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bOFull + t * NS + gp % NS),
+                                                     (gp / NS) & 1u, &g_fa_error, p.timeout_ns));
+              if (!ok) break;
+              tc_fence_after();
+            }
+            const float f = need ? ex2_approx((m_ref - m_new) * sl2) : 1.f;
+            if (need) {
+              l *= f;
+              m_ref = m_new;
+            }
+            const uint32_t o_addr = tmem + lane_addr + C::o_col(t);
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t r[32];
+              tmem_ld32(o_addr + 32 * c, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
+              tmem_st32(o_addr + 32 * c, r);
+            }
+            tmem_wait_st();
+          }
+        }
+        const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * sl2;
+        float lsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          s[c] = ex2_approx(fmaf(s[c], sl2, -mc));
+          lsum += s[c];
+        }
+        l += lsum;
+#pragma unroll
+        for (int c = 0; c < BN / 64; ++c) {
+          uint32_t r[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = pack2<C::HALF>(s[64 * c + 2 * e], s[64 * c + 2 * e + 1]);
+          tmem_st32(s_addr + 32 * c, r);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      mbar_arrive(bar(C::bPFull + t * NS + buf));
+    }
+    if (!ok) break;
+
+    // epilogue
+    const float inv_l = l > 0.f ? 1.f / l : 0.f;
+    const float lse_v = l > 0.f ? (m_ref * sl2 + lg2_approx(l)) * 0.69314718055994531f : -INFINITY;
+    const size_t orow = (size_t)(U.q_start + i) * p.Hq + h;  // packed (token, head) row
+    if (U.nb > 0) {
+      const uint32_t gl = s_cnt + U.nb - 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bOFull + t * NS + gl % NS), (gl / NS) & 1u,
+                                             &g_fa_error, p.timeout_ns));
+      if (!ok) break;
+      tc_fence_after();
+    }
+    if (warp_on) {
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        if (U.nb > 0) {
+          tmem_ld32(tmem + lane_addr + C::o_col(t) + 32 * c, r);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = 0u;
+        }
+        if (valid) {
+          if constexpr (C::PARTIAL) {
+            float *dst = p.o_part + ((size_t)U.split * p.total_q * p.Hq + orow) * D + 32 * c;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              float4 w = make_float4(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l,
+                                     __uint_as_float(r[e + 2]) * inv_l,
+                                     __uint_as_float(r[e + 3]) * inv_l);
+              *reinterpret_cast<float4 *>(dst + e) = w;
+            }
+          } else {
+            uint16_t *dst = reinterpret_cast<uint16_t *>(p.out) + orow * D + 32 * c;
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint4 w;
+              w.x = pack2<C::HALF>(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l);
+              w.y = pack2<C::HALF>(__uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
+              w.z = pack2<C::HALF>(__uint_as_float(r[e + 4]) * inv_l, __uint_as_float(r[e + 5]) * inv_l);
+              w.w = pack2<C::HALF>(__uint_as_float(r[e + 6]) * inv_l, __uint_as_float(r[e + 7]) * inv_l);
+              *reinterpret_cast<uint4 *>(dst + e) = w;
+            }
+          }
+        }
+      }
+    }
+    if (valid) {
+      if constexpr (C::PARTIAL) {
+        p.lse_part[(size_t)U.split * p.total_q * p.Hq + orow] = lse_v;
+      } else if (p.lse != nullptr) {
+        const size_t li = p.lse_dense ? ((size_t)U.b * p.Hq + h) * p.Sq + i
+                                      : (size_t)h * p.total_q + U.q_start + i;
+        p.lse[li] = lse_v;
+      }
+    }
+    if (U.nb > 0) {
+      tc_fence_before();
+      mbar_arrive(bar(C::bOEmpty + t));
+    }
+    s_cnt += U.nb;
+  }
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::kThreads, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int warp = warp_id_sync();
+  const int lane = threadIdx.x & 31;
+
+  if (warp == 0 && lane == 0) {
+    for (int b = 0; b < C::kNumBars; ++b) {
+      uint32_t cnt = 1;
+      if (b >= C::bPFull && b < C::bPFull + C::NQ * C::NS) cnt = 128;
+      if (b >= C::bOEmpty && b < C::bOEmpty + C::NQ) cnt = 128;
+      mbar_init(sb + C::kBarOff + 8u * b, cnt);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&p.tm_q);
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(sb + C::kSlotOff, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + C::kSlotOff);
+
+  if (warp == 0) {
+    if (lane == 0) role_producer<C>(p, sb);
+  } else if (warp == 1) {
+    if (lane == 0) role_mma<C>(p, sb, tmem);
+  } else if (warp >= 4) {
+    role_softmax<C>(p, sb, tmem, warp / 4 - 1);
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// split-KV merge: one warp per packed (token, head) row
+// ---------------------------------------------------------------------------
+template <int D, bool HALF>
+__global__ void __launch_bounds__(256) fa_combine_kernel(const float *__restrict__ o_part,
+                                                         const float *__restrict__ lse_part,
+                                                         int ns, long long rows, void *out,
+                                                         float *lse, int Hq, int Sq,
+                                                         int total_q, int lse_dense) {
+  constexpr int E = D / 32;  // elements per lane
+  const long long r = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const float L2E = 1.4426950408889634f;
+  float m = -INFINITY;
+  for (int s = lane; s < ns; s += 32) m = fmaxf(m, lse_part[(long long)s * rows + r]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float z = 0.f;
+  if (m != -INFINITY)
+    for (int s = lane; s < ns; s += 32) z += ex2_approx((lse_part[(long long)s * rows + r] - m) * L2E);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  const float Lse = (m == -INFINITY) ? -INFINITY : m + lg2_approx(z) * 0.69314718055994531f;
+  float acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  if (m != -INFINITY) {
+    for (int s = 0; s < ns; ++s) {
+      const float ls = lse_part[(long long)s * rows + r];
+      if (ls == -INFINITY) continue;
+      const float w = ex2_approx((ls - Lse) * L2E);
+      const float *src = o_part + ((long long)s * rows + r) * D + lane * E;
+#pragma unroll
+      for (int e = 0; e < E; e += 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(src + e);
+        acc[e] += w * x.x;
+        acc[e + 1] += w * x.y;
+        acc[e + 2] += w * x.z;
+        acc[e + 3] += w * x.w;
+      }
+    }
+  }
+  uint16_t *dst = reinterpret_cast<uint16_t *>(out) + r * D + lane * E;
+#pragma unroll
+  for (int e = 0; e < E; e += 4) {
+    uint2 w;
+    w.x = pack2<HALF>(acc[e], acc[e + 1]);
+    w.y = pack2<HALF>(acc[e + 2], acc[e + 3]);
+    *reinterpret_cast<uint2 *>(dst + e) = w;
+  }
+  if (lane == 0 && lse != nullptr) {
+    const long long tok = r / Hq;
+    const int h = (int)(r % Hq);
+    const long long li =
+        lse_dense ? ((tok / Sq) * Hq + h) * (long long)Sq + tok % Sq : (long long)h * total_q + tok;
+    lse[li] = Lse;
+  }
+}
+
+}  // namespace fab

@@ -39,16 +39,16 @@ WORKLOADS = ["dense_257", "varlen_gqa_bias", "video_dit_20480",
 _CHUNK = 1 << 24
 
 
-def _randn(shape, gen: torch.Generator, dtype, std: float = 1.0,
-           device="cpu") -> torch.Tensor:
-    """N(0, std^2) in float32, rounded to ``dtype``, drawn in chunks."""
+def _randn(shape, gen: torch.Generator, dtype, std: float = 1.0) -> torch.Tensor:
+    """N(0, std^2) in float32, rounded to ``dtype``, drawn in chunks on the
+    generator's device."""
     n = 1
     for s in shape:
         n *= int(s)
-    out = torch.empty(n, dtype=dtype, device=device)
+    out = torch.empty(n, dtype=dtype, device=gen.device)
     for start in range(0, n, _CHUNK):
         m = min(_CHUNK, n - start)
-        x = torch.randn(m, generator=gen, dtype=torch.float32)
+        x = torch.randn(m, generator=gen, dtype=torch.float32, device=gen.device)
         if std != 1.0:
             x.mul_(std)
         out[start:start + m].copy_(x)
@@ -142,10 +142,15 @@ class Problem:
                        dict(self.meta))
 
 
-def make(name: str, dtype=torch.bfloat16) -> Problem:
-    """Build one named workload with its fixed seed."""
+def make(name: str, dtype=torch.bfloat16, device="cpu") -> Problem:
+    """Build one named workload with its fixed seed.
+
+    With ``device`` other than the CPU the values are drawn there by that
+    device's seeded generator (another stream of numbers than the CPU
+    generator's, same distributions and shapes): the benchmark uses this for
+    the multi-GB workloads; parity tests draw on the CPU."""
     idx = WORKLOADS.index(name)
-    g = torch.Generator().manual_seed(SEED_BASE + idx)
+    g = torch.Generator(device=device).manual_seed(SEED_BASE + idx)
     if name == "dense_257":
         B, S, H, D = 1, 257, 8, 128
         q = _randn((B, S, H, D), g, dtype)
@@ -155,8 +160,8 @@ def make(name: str, dtype=torch.bfloat16) -> Problem:
                        max_seqlen_q=S, max_seqlen_k=S)
     if name == "varlen_gqa_bias":
         Hq, Hkv, D, R = 32, 8, 128, 256
-        lens = torch.randint(512, 4097, (4,), generator=g).tolist()
-        cu = torch.tensor([0] + list(_cumsum(lens)), dtype=torch.int32)
+        lens = torch.randint(512, 4097, (4,), generator=g, device=g.device).tolist()
+        cu = torch.tensor([0] + list(_cumsum(lens)), dtype=torch.int32, device=g.device)
         total = int(cu[-1])
         q = _randn((total, Hq, D), g, dtype)
         k = _randn((total, Hkv, D), g, dtype)
@@ -181,7 +186,7 @@ def make(name: str, dtype=torch.bfloat16) -> Problem:
         v = _randn((B, Sk, Hkv, D), g, dtype)
         k[:, used:] = 1e4
         v[:, used:] = 1e4
-        su = torch.full((B,), used, dtype=torch.int32)
+        su = torch.full((B,), used, dtype=torch.int32, device=g.device)
         return Problem(name, "dense", q, k, v, softmax_scale=1 / math.sqrt(D),
                        seqused_k=su, max_seqlen_q=Sq, max_seqlen_k=Sk)
     if name == "decode_splitkv":

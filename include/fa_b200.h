@@ -1,0 +1,153 @@
+/*
+ * fa_b200.h -- exact attention forward for B200 (sm_100a), C ABI.
+ *
+ * Computes, for every query row of every head,
+ *
+ *     O   = softmax(scale * Q K^T + bias + mask) V
+ *     LSE = log( sum_j exp(scale * q.k_j + bias_j) )   (natural log, fp32)
+ *
+ * tile by tile with an online softmax, so the score matrix never reaches
+ * device memory.  The operation and its arguments follow these passages of
+ * the source pages:
+ *
+ *   - "FlashAttention-4" (H3 runtime), API: [batch, sequence, heads, head_dim]
+ *     layout, matching fp16/bf16 Q/K/V, and an error instead of a silent
+ *     change of kernel for anything unsupported.
+ *   - "flashrt/fa4-cute-runtime", Functions: the forward returns (out, lse);
+ *     forward_static writes into a caller-preallocated out; seqused_k is a
+ *     device int32 tensor holding the valid K/V length of a padded buffer;
+ *     pack_gqa packs the query heads that share one K/V head.
+ *   - "mgoin/tml-fa4", argument contract: varlen q [total_q, Hq, D],
+ *     k/v [total_k, Hkv, D], cu_seqlens int32 [B+1] whose last entry is the
+ *     total; rel_bias [total_q, Hq, rel_extent] in q's order and dtype with
+ *     rel_extent a multiple of 128; the distance d = i + (k_len - q_len) - j,
+ *     score += rel_bias[cu_seqlens_q[b] + i, h, d] when 0 <= d < rel_extent;
+ *     in causal mode d == 0 is the query's own key (keys with d < 0 masked).
+ *   - "mgoin/tml-fa4" (split-KV combine) and "FlashAttention-4 backend for
+ *     Blackwell #1235" (split over keys merged through the LSE): the
+ *     split-KV entry point.
+ *
+ * Conventions shared by every entry point
+ *   - All pointers are DEVICE pointers of the current CUDA device, owned by
+ *     the caller.  The library allocates no device memory and never
+ *     synchronises the stream: a call only enqueues work on `stream`
+ *     (a cudaStream_t; NULL means the legacy default stream) and returns.
+ *   - Element type `dt` applies to q, k, v, out and rel_bias alike.
+ *   - head_dim D must be 128 or 256; Hq must be a multiple of Hkv; query head
+ *     h reads K/V head h / (Hq / Hkv).
+ *   - q, k, v, out and rel_bias must be 16-byte aligned and contiguous in the
+ *     documented layout.  cu_seqlens and seqused_k are device int32 arrays.
+ *   - softmax_scale <= 0 selects 1 / sqrt(D).
+ *   - A query row with no admissible key gets O = 0 and LSE = -inf.
+ *   - K/V rows that a call reads but masks (beyond seqused_k, or the padding
+ *     of a ragged tile) must hold finite values.
+ *   - Errors: invalid arguments return FA_ERR_INVALID or FA_ERR_UNSUPPORTED
+ *     before anything is enqueued; a launch failure returns FA_ERR_CUDA.  No
+ *     entry point ever falls back to another algorithm.  A message for the
+ *     last failure of the calling thread is available from
+ *     fa_last_error_message().
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID = 1,        /* malformed arguments (null, shape, alignment) */
+  FA_ERR_UNSUPPORTED = 2,    /* well-formed but not served (e.g. D = 64)    */
+  FA_ERR_CUDA = 3,           /* a CUDA runtime call or launch failed         */
+  FA_ERR_WORKSPACE = 4,      /* split-KV workspace missing or too small      */
+  FA_ERR_DEVICE_TIMEOUT = 5  /* a kernel gave up waiting (see below)         */
+} fa_status;
+
+typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
+
+/*
+ * Dense forward.
+ *   q   [B, Sq, Hq, D]    k, v [B, Sk, Hkv, D]    out [B, Sq, Hq, D]
+ *   lse [B, Hq, Sq] float32 (may be NULL when not wanted)
+ *   causal: bottom-right aligned (key j admitted iff j <= i + k_len - Sq).
+ *   seqused_k: NULL, or device int32 [B] with 0 <= seqused_k[b] <= Sk; batch
+ *     entry b then uses keys [0, seqused_k[b]) of its padded K/V rows and
+ *     k_len = seqused_k[b] in the causal and bias distance.
+ *   rel_bias: NULL, or [B*Sq, Hq, rel_extent] in q's dtype (the dense form of
+ *     the varlen layout, rows in q's flattened order), rel_extent % 128 == 0.
+ */
+fa_status fa_fwd(const void *q, const void *k, const void *v, void *out,
+                 float *lse, int B, int Sq, int Sk, int Hq, int Hkv, int D,
+                 fa_dtype dt, int causal, float softmax_scale,
+                 const int *seqused_k, const void *rel_bias, int rel_extent,
+                 void *stream);
+
+/*
+ * Variable-length forward ("mgoin/tml-fa4", argument contract).
+ *   q [total_q, Hq, D]   k, v [total_k, Hkv, D]   out [total_q, Hq, D]
+ *   lse [Hq, total_q] float32 (may be NULL)
+ *   cu_seqlens_q, cu_seqlens_k: device int32 [B+1], nondecreasing, first 0,
+ *     last total_q / total_k.
+ *   max_seqlen_q: the largest q length (sizes the launch; rows of a longer
+ *     sequence are not computed).  max_seqlen_k is accepted for API parity.
+ *   seqused_k: NULL or device int32 [B]; k_len_b = seqused_k[b] (at most the
+ *     cu_seqlens_k length).
+ *   rel_bias: NULL or [total_q, Hq, rel_extent], rel_extent % 128 == 0.
+ */
+fa_status fa_fwd_varlen(const void *q, const void *k, const void *v, void *out,
+                        float *lse, const int *cu_seqlens_q,
+                        const int *cu_seqlens_k, const int *seqused_k, int B,
+                        int max_seqlen_q, int max_seqlen_k, int total_q,
+                        int total_k, int Hq, int Hkv, int D, fa_dtype dt,
+                        int causal, float softmax_scale, const void *rel_bias,
+                        int rel_extent, void *stream);
+
+/*
+ * Split-KV forward (decode): keys are cut into num_splits contiguous ranges,
+ * each range yields a float32 partial (O normalised over the range, and its
+ * LSE) in `workspace`, and a second kernel merges them through the LSE:
+ *     lse = log sum_s exp(lse_s),   O = sum_s exp(lse_s - lse) O_s.
+ * Arguments as fa_fwd, plus:
+ *   num_splits: 0 picks fa_splitkv_default_splits(); otherwise >= 1 (the
+ *     effective count can be lower when the ranges, rounded to whole key
+ *     tiles, cover Sk sooner).
+ *   workspace: device memory of at least fa_splitkv_workspace_bytes(...)
+ *     bytes, 16-byte aligned, owned by the caller; its contents on entry do
+ *     not matter and are overwritten.
+ */
+size_t fa_splitkv_workspace_bytes(int B, int Sq, int Hq, int D, int num_splits);
+int fa_splitkv_default_splits(int B, int Sq, int Sk, int Hq, int Hkv, int D,
+                              int num_sms);
+fa_status fa_fwd_splitkv(const void *q, const void *k, const void *v, void *out,
+                         float *lse, int B, int Sq, int Sk, int Hq, int Hkv,
+                         int D, fa_dtype dt, int causal, float softmax_scale,
+                         const int *seqused_k, const void *rel_bias,
+                         int rel_extent, int num_splits, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
+/*
+ * Device-side watchdog.  Every wait inside the kernels is bounded; a kernel
+ * that gives up records a code in a device word and returns without
+ * trapping.  This call synchronises the current device, copies that word to
+ * *code (0 = none) and, if clear != 0, resets it.  Returns FA_OK, or
+ * FA_ERR_DEVICE_TIMEOUT when the word was set, or FA_ERR_CUDA.
+ */
+fa_status fa_check_device_error(int *code, int clear);
+
+/* Human-readable name of a status; never NULL. */
+const char *fa_status_string(fa_status s);
+
+/* Message for the calling thread's last failed call ("" if none). */
+const char *fa_last_error_message(void);
+
+/* Library version string. */
+const char *fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

@@ -1,0 +1,71 @@
+"""Element-wise comparison of the CUDA path against the fp64 oracle.
+
+Gates (stated for this operation): on O, max-abs <= 1e-2 and mean-abs <= 5e-4
+for bf16 and fp16 outputs; on the LSE, |dLSE| <= 1e-3 * max(1, |LSE|).  The
+relative RMS error of O (<= 1e-2) is also checked, because with N(0,1) inputs
+and long key ranges |O| is so small that the absolute gates say little.
+Rows with no admissible key must give O == 0 exactly and LSE == -inf.
+"""
+import math
+
+import numpy as np
+import torch
+
+MAX_ABS = 1e-2
+MEAN_ABS = 5e-4
+LSE_REL = 1e-3
+REL_RMS = 1e-2
+
+
+def to_np(t):
+    if isinstance(t, torch.Tensor):
+        return t.detach().float().cpu().numpy().astype(np.float64)
+    return np.asarray(t, dtype=np.float64)
+
+
+def compare(out, lse, ref_o, ref_l, *, max_abs=MAX_ABS, mean_abs=MEAN_ABS,
+            lse_rel=LSE_REL, rel_rms=REL_RMS, what=""):
+    stats = {}
+    if out is not None:
+        o = to_np(out).reshape(ref_o.shape)
+        ref_o = np.asarray(ref_o, dtype=np.float64)
+        err = np.abs(o - ref_o)
+        stats["max_abs"] = float(err.max()) if err.size else 0.0
+        stats["mean_abs"] = float(err.mean()) if err.size else 0.0
+        assert np.isfinite(o).all(), f"{what}: non-finite output"
+        assert stats["max_abs"] <= max_abs, f"{what}: {stats}"
+        assert stats["mean_abs"] <= mean_abs, f"{what}: {stats}"
+        nrm = float(np.sqrt((ref_o ** 2).sum()))
+        if nrm > 0:
+            stats["rel_rms"] = float(np.sqrt((err ** 2).sum())) / nrm
+            assert stats["rel_rms"] <= rel_rms, f"{what}: {stats}"
+    if lse is not None:
+        l = to_np(lse).reshape(ref_l.shape)
+        ref_l = np.asarray(ref_l, dtype=np.float64)
+        inf = np.isneginf(ref_l)
+        assert (np.isneginf(l) == inf).all(), f"{what}: -inf LSE pattern differs"
+        fin = ~inf
+        if fin.any():
+            d = np.abs(l[fin] - ref_l[fin]) / np.maximum(1.0, np.abs(ref_l[fin]))
+            stats["lse_rel"] = float(d.max())
+            assert stats["lse_rel"] <= lse_rel, f"{what}: {stats}"
+    return stats
+
+
+def lse_rows(lse_dense_bhs, rows):
+    """Pick LSE values [B,Hq,Sq] at rows (b, h, i)."""
+    l = to_np(lse_dense_bhs)
+    return np.array([l[b, h, i] for b, h, i in rows])
+
+
+def compare_relative(out, ref_o, *, ulps=2.0, floor=2e-3, what=""):
+    """Stress inputs (sharp softmax, large bias or offset values): |O| reaches
+    several units, where one bf16 ulp alone exceeds the absolute gate.  Gate
+    each element at `ulps` bf16 ulps of the reference plus a small floor."""
+    o = to_np(out).reshape(np.shape(ref_o))
+    ref_o = np.asarray(ref_o, dtype=np.float64)
+    err = np.abs(o - ref_o)
+    bound = ulps * np.abs(ref_o) * 2.0 ** -8 + floor
+    worst = float((err / bound).max()) if err.size else 0.0
+    assert worst <= 1.0, f"{what}: worst err/bound {worst:.3f}, max_abs {err.max():.4g}"
+    return worst

@@ -1,0 +1,112 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+The library must load, export every entry point that include/fa_b200.h
+declares, and reject malformed arguments with a status before it touches the
+device -- never by falling back to another computation.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_attention_forward_flash_b200 as fa
+from exact_attention_forward_flash_b200 import build as fa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa_b200.h")
+
+FA_OK, FA_ERR_INVALID, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_WORKSPACE = 0, 1, 2, 3, 4
+
+# a 16-byte aligned address that the library never dereferences in these
+# tests (every call below fails validation first)
+A = ctypes.c_void_p(0x10000)
+MIS = ctypes.c_void_p(0x10008)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fa_build.build()
+    return fa.load_library()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_entry_point(lib):
+    names = _declared()
+    assert {"fa_fwd", "fa_fwd_varlen", "fa_fwd_splitkv"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError):
+        fa.load_library(str(tmp_path / "nope.so"))
+
+
+def _fwd(lib, q=A, k=A, v=A, out=A, lse=A, B=1, Sq=16, Sk=16, Hq=4, Hkv=2, D=128,
+         dt=0, causal=0, scale=0.0, su=None, rb=None, R=0):
+    return lib.fa_fwd(q, k, v, out, lse, B, Sq, Sk, Hq, Hkv, D, dt, causal, scale,
+                      su, rb, R, None)
+
+
+def test_validation_statuses(lib):
+    assert _fwd(lib, D=64) == FA_ERR_UNSUPPORTED
+    assert _fwd(lib, D=192) == FA_ERR_UNSUPPORTED
+    assert _fwd(lib, Hq=6, Hkv=4) == FA_ERR_INVALID
+    assert _fwd(lib, dt=7) == FA_ERR_INVALID
+    assert _fwd(lib, q=None) == FA_ERR_INVALID
+    assert _fwd(lib, k=None) == FA_ERR_INVALID
+    assert _fwd(lib, q=MIS) == FA_ERR_INVALID
+    assert _fwd(lib, out=MIS) == FA_ERR_INVALID
+    assert _fwd(lib, rb=A, R=100) == FA_ERR_INVALID      # rel_extent % 128
+    assert _fwd(lib, rb=A, R=0) == FA_ERR_INVALID
+    assert _fwd(lib, rb=MIS, R=128) == FA_ERR_INVALID
+    assert _fwd(lib, scale=float("nan")) == FA_ERR_INVALID
+    assert _fwd(lib, Sq=-1) == FA_ERR_INVALID
+    assert _fwd(lib, B=-1) == FA_ERR_INVALID
+    msg = lib.fa_last_error_message().decode()
+    assert msg, "a failed call leaves a message"
+
+
+def test_empty_problems_are_no_ops(lib):
+    # nothing to compute: success without touching the device
+    assert _fwd(lib, B=0) == FA_OK
+    assert _fwd(lib, Sq=0) == FA_OK
+
+
+def test_varlen_validation(lib):
+    P = None
+    r = lib.fa_fwd_varlen(A, A, A, A, A, None, None, None, 2, 8, 8, 16, 16, 4, 2,
+                          128, 0, 0, 0.0, None, 0, None)
+    assert r == FA_ERR_INVALID  # cu_seqlens missing
+    r = lib.fa_fwd_varlen(A, A, A, A, A, A, A, P, 2, 8, 8, 16, 16, 4, 2, 64, 0, 0,
+                          0.0, None, 0, None)
+    assert r == FA_ERR_UNSUPPORTED
+
+
+def test_splitkv_host_logic(lib):
+    ws = lib.fa_splitkv_workspace_bytes
+    assert ws(8, 1, 32, 128, 37) >= 37 * 8 * 32 * 129 * 4
+    assert ws(8, 1, 32, 128, 37) % 256 == 0
+    assert ws(0, 1, 32, 128, 4) == 0
+    ds = lib.fa_splitkv_default_splits
+    # 8 x 8 (batch, K/V head) units of one tile each on 148 SMs: split for
+    # about 16 units per SM, every split at least 8 key tiles long
+    ns = ds(8, 1, 131072, 32, 8, 128, 148)
+    assert 16 <= ns <= 256
+    assert ds(8, 1, 2048, 32, 8, 128, 148) <= 2            # short keys
+    assert ds(64, 1024, 4096, 32, 32, 128, 148) == 1        # already many units
+    r = lib.fa_fwd_splitkv(A, A, A, A, A, 1, 1, 16, 4, 2, 128, 0, 0, 0.0, None,
+                           None, 0, -1, A, 1 << 20, None)
+    assert r == FA_ERR_INVALID
+
+
+def test_status_strings(lib):
+    for s, name in [(0, "FA_OK"), (1, "FA_ERR_INVALID"), (2, "FA_ERR_UNSUPPORTED"),
+                    (3, "FA_ERR_CUDA"), (4, "FA_ERR_WORKSPACE"), (5, "FA_ERR_DEVICE_TIMEOUT")]:
+        assert lib.fa_status_string(s).decode() == name

@@ -1,0 +1,316 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU fp64 oracle.
+
+Every case draws seeded inputs from fa_inputs, runs the library on cuda:0 and
+compares element by element (tests/parity_util.py states the gates).  Sizes
+span several tiles and a ragged tail; the full-size workloads are checked on
+sampled rows, which the oracle computes one by one exactly.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import fa_inputs
+import oracle
+import exact_attention_forward_flash_b200 as fa
+from parity_util import compare, compare_relative, to_np
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    fa.load_library()
+    yield
+    assert fa.check_device_error() == 0, "a kernel wait timed out"
+
+
+def run_dense(p, **kw):
+    g = p.to(DEV)
+    out, lse = fa.fa_fwd(g.q, g.k, g.v, causal=p.causal, softmax_scale=p.softmax_scale,
+                         seqused_k=g.seqused_k, rel_bias=g.rel_bias, **kw)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+def ref_dense(p):
+    return oracle.attention(p.q, p.k, p.v, causal=p.causal, softmax_scale=p.softmax_scale,
+                            seqused_k=p.seqused_k, rel_bias=p.rel_bias)
+
+
+def run_varlen(p):
+    g = p.to(DEV)
+    out, lse = fa.fa_fwd_varlen(g.q, g.k, g.v, g.cu_seqlens_q, g.cu_seqlens_k,
+                                p.max_seqlen_q, p.max_seqlen_k, seqused_k=g.seqused_k,
+                                causal=p.causal, softmax_scale=p.softmax_scale,
+                                rel_bias=g.rel_bias)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+def ref_varlen(p):
+    return oracle.attention(p.q, p.k, p.v, cu_seqlens_q=p.cu_seqlens_q,
+                            cu_seqlens_k=p.cu_seqlens_k, seqused_k=p.seqused_k,
+                            causal=p.causal, softmax_scale=p.softmax_scale,
+                            rel_bias=p.rel_bias)
+
+
+# ---------------------------------------------------------------------------
+# the small dense workload, both 16-bit types
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_dense_257(dtype):
+    p = fa_inputs.make("dense_257", dtype=dtype)
+    out, lse = run_dense(p)
+    ro, rl = ref_dense(p)
+    compare(out, lse, ro, rl, what=f"dense_257 {dtype}")
+
+
+# ---------------------------------------------------------------------------
+# dense shapes: causal, Sq != Sk both ways, GQA groups, D = 128 / 256
+# ---------------------------------------------------------------------------
+CASES = [
+    # B, Sq, Sk, Hq, Hkv, D, causal
+    (2, 300, 300, 4, 4, 128, True),
+    (1, 300, 200, 4, 2, 128, True),    # k shorter: first rows see no key
+    (1, 100, 333, 8, 2, 128, True),    # k longer: bottom-right diagonal
+    (2, 129, 390, 6, 2, 128, False),   # group of 3: heads not packed
+    (1, 257, 257, 16, 2, 128, True),   # group of 8 packed
+    (2, 200, 300, 8, 8, 256, False),
+    (1, 300, 300, 8, 1, 256, True),    # D=256, group of 8 packed
+    (1, 70, 600, 4, 4, 256, True),
+]
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_dense_shapes(case):
+    B, Sq, Sk, Hq, Hkv, D, causal = case
+    p = fa_inputs.random_dense(100 + Sq + Sk, B, Sq, Sk, Hq, Hkv, D, causal=causal)
+    out, lse = run_dense(p)
+    ro, rl = ref_dense(p)
+    compare(out, lse, ro, rl, what=str(case))
+
+
+@pytest.mark.parametrize("D", [128, 256])
+def test_fp16_causal_gqa(D):
+    p = fa_inputs.random_dense(7, 2, 260, 270, 8, 2, D, dtype=torch.float16, causal=True)
+    out, lse = run_dense(p)
+    ro, rl = ref_dense(p)
+    compare(out, lse, ro, rl, what=f"fp16 D{D}")
+
+
+# ---------------------------------------------------------------------------
+# varlen with empty / one-token / multi-tile sequences, causal, GQA, bias
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("D", [128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_bias(D, causal):
+    q_lens = [0, 1, 130, 257, 513, 64]
+    k_lens = [3, 1, 130, 300, 513, 0]
+    p = fa_inputs.random_varlen(11 + D, q_lens, k_lens, Hq=8, Hkv=2, D=D, causal=causal,
+                                bias_extent=256)
+    out, lse = run_varlen(p)
+    ro, rl = ref_varlen(p)
+    compare(out, lse, ro, rl, what=f"varlen D{D} causal={causal}")
+
+
+def test_varlen_seqused():
+    p = fa_inputs.random_varlen(12, [100, 200], [300, 250], Hq=4, Hkv=4, D=128, causal=True,
+                                seqused=[260, 250], bias_extent=128)
+    out, lse = run_varlen(p)
+    ro, rl = ref_varlen(p)
+    compare(out, lse, ro, rl, what="varlen seqused")
+
+
+def test_bias_extent_512_far_band():
+    # rel_extent larger than one KV tile and q_len < k_len
+    p = fa_inputs.random_varlen(13, [200, 333], [700, 333], Hq=4, Hkv=1, D=128, causal=True,
+                                bias_extent=512, bias_std=0.5)
+    out, lse = run_varlen(p)
+    ro, rl = ref_varlen(p)
+    compare(out, lse, ro, rl, what="bias 512")
+    # a strong bias (std 2) sharpens the rows: gate on relative error
+    p = fa_inputs.random_varlen(14, [200, 333], [700, 333], Hq=4, Hkv=1, D=128, causal=True,
+                                bias_extent=512, bias_std=2.0)
+    out, lse = run_varlen(p)
+    ro, rl = ref_varlen(p)
+    compare(None, lse, ro, rl, max_abs=1.0, mean_abs=1.0, rel_rms=1.0, what="bias 512 std 2 lse")
+    compare_relative(out, ro, what="bias 512 std 2")
+
+
+# ---------------------------------------------------------------------------
+# the padded D=256 encoder workload (seqused_k, padding holds 1e4), in full
+# ---------------------------------------------------------------------------
+def test_encoder_d256_seqused():
+    p = fa_inputs.make("encoder_d256_seqused")
+    out, lse = run_dense(p)
+    ro, rl = ref_dense(p)
+    compare(out, lse, ro, rl, what="encoder_d256_seqused")
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads on sampled rows
+# ---------------------------------------------------------------------------
+def _sample_rows(rng, B, Hq, lens, n):
+    rows = []
+    for _ in range(n):
+        b = int(rng.integers(B))
+        L = lens[b]
+        i = int(rng.choice([0, L - 1, int(rng.integers(L)), min(L - 1, 127), min(L - 1, 128)]))
+        rows.append((b, int(rng.integers(Hq)), i))
+    return np.array(rows, dtype=np.int32)
+
+
+def test_varlen_gqa_bias_workload_sampled():
+    p = fa_inputs.make("varlen_gqa_bias")
+    out, lse = run_varlen(p)
+    lens = p.meta["lens"]
+    rows = _sample_rows(np.random.default_rng(0), 4, 32, lens, 512)
+    ro, rl = oracle.attention_rows(p.q, p.k, p.v, rows, cu_seqlens_q=p.cu_seqlens_q,
+                                   cu_seqlens_k=p.cu_seqlens_k, causal=True,
+                                   softmax_scale=p.softmax_scale, rel_bias=p.rel_bias)
+    cq = p.cu_seqlens_q.tolist()
+    o = out.float().cpu()
+    l = lse.cpu()
+    go = np.stack([o[cq[b] + i, h].numpy() for b, h, i in rows])
+    gl = np.array([float(l[h, cq[b] + i]) for b, h, i in rows])
+    compare(go, gl, ro, rl, what="varlen_gqa_bias sampled")
+
+
+def test_video_dit_20480_sampled():
+    p = fa_inputs.make("video_dit_20480")
+    out, lse = run_dense(p)
+    rows = _sample_rows(np.random.default_rng(1), 1, 56, [20480], 256)
+    ro, rl = oracle.attention_rows(p.q, p.k, p.v, rows, softmax_scale=p.softmax_scale)
+    o = out.float().cpu()
+    l = lse.cpu()
+    go = np.stack([o[b, i, h].numpy() for b, h, i in rows])
+    gl = np.array([float(l[b, h, i]) for b, h, i in rows])
+    compare(go, gl, ro, rl, what="video_dit sampled")
+
+
+# ---------------------------------------------------------------------------
+# split-KV
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("ns", [0, 1, 3, 7])
+@pytest.mark.parametrize("D", [128, 256])
+def test_splitkv_small(ns, D):
+    p = fa_inputs.random_dense(21 + D, 3, 1, 1000, 8, 2, D)
+    g = p.to(DEV)
+    out, lse = fa.fa_fwd_splitkv(g.q, g.k, g.v, num_splits=ns)
+    torch.cuda.synchronize()
+    ro, rl = ref_dense(p)
+    compare(out, lse, ro, rl, what=f"splitkv ns={ns} D={D}")
+
+
+def test_splitkv_causal_multi_query_seqused():
+    p = fa_inputs.random_dense(22, 2, 5, 900, 8, 2, 128, causal=True, seqused=[700, 900],
+                               pad_value=1e4, bias_extent=128)
+    g = p.to(DEV)
+    out, lse = fa.fa_fwd_splitkv(g.q, g.k, g.v, num_splits=5, causal=True,
+                                 seqused_k=g.seqused_k, rel_bias=g.rel_bias)
+    torch.cuda.synchronize()
+    ro, rl = ref_dense(p)
+    compare(out, lse, ro, rl, what="splitkv causal seqused bias")
+
+
+def test_decode_splitkv_workload():
+    p = fa_inputs.make("decode_splitkv")
+    g = p.to(DEV)
+    out, lse = fa.fa_fwd_splitkv(g.q, g.k, g.v, softmax_scale=p.softmax_scale)
+    torch.cuda.synchronize()
+    del g
+    o = out.float().cpu()
+    l = lse.cpu()
+    for b in range(p.B):  # one batch entry at a time keeps host memory small
+        ro, rl = oracle.attention(p.q[b:b + 1], p.k[b:b + 1], p.v[b:b + 1],
+                                  softmax_scale=p.softmax_scale)
+        compare(o[b:b + 1], l[b:b + 1], ro, rl, what=f"decode b={b}")
+
+
+# ---------------------------------------------------------------------------
+# edge cases and invariants
+# ---------------------------------------------------------------------------
+def test_no_keys_gives_zero_and_minus_inf():
+    p = fa_inputs.random_dense(30, 2, 40, 50, 4, 2, 128, seqused=[0, 50])
+    out, lse = run_dense(p)
+    ro, rl = ref_dense(p)
+    compare(out, lse, ro, rl, what="seqused 0")
+    assert (out[0] == 0).all() and torch.isneginf(lse[0]).all()
+
+
+def test_zero_length_keys_everywhere():
+    p = fa_inputs.random_dense(31, 1, 10, 0, 2, 2, 128)
+    g = p.to(DEV)
+    out, lse = fa.fa_fwd(g.q, g.k, g.v)
+    torch.cuda.synchronize()
+    assert (out == 0).all() and torch.isneginf(lse).all()
+
+
+def test_empty_batch_is_a_no_op():
+    q = torch.empty((0, 5, 2, 128), dtype=torch.bfloat16, device=DEV)
+    out, lse = fa.fa_fwd(q, q, q)
+    torch.cuda.synchronize()
+    assert out.numel() == 0
+
+
+def test_bias_none_equals_bias_zero_bitwise():
+    p = fa_inputs.random_dense(32, 1, 300, 300, 4, 4, 128, causal=True)
+    g = p.to(DEV)
+    o1, l1 = fa.fa_fwd(g.q, g.k, g.v, causal=True)
+    zb = torch.zeros((300, 4, 128), dtype=torch.bfloat16, device=DEV)
+    o2, l2 = fa.fa_fwd(g.q, g.k, g.v, causal=True, rel_bias=zb)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_deterministic_run_to_run():
+    p = fa_inputs.random_varlen(33, [500, 129], [700, 129], Hq=8, Hkv=2, D=128, causal=True,
+                                bias_extent=256)
+    o1, l1 = run_varlen(p)
+    o2, l2 = run_varlen(p)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_stress_peaked_and_offset_values():
+    # sharp softmax (q * 8) and values far from zero (V + 4): bf16 rounding of
+    # O near 4 is ~0.016, so this case is gated on relative error
+    p = fa_inputs.random_dense(34, 1, 256, 384, 4, 2, 128, causal=True, q_std=8.0,
+                               v_offset=4.0)
+    out, lse = run_dense(p)
+    ro, rl = ref_dense(p)
+    compare(None, lse, ro, rl, max_abs=1.0, mean_abs=1.0, rel_rms=1.0, what="stress lse")
+    compare_relative(out, ro, what="stress")
+
+
+def test_many_batches_beyond_grid_y_limit():
+    # batch x heads well past 65535 (the grid-dimension limit a kernel that
+    # put them in gridDim.y would hit)
+    B = 70000
+    p = fa_inputs.random_dense(35, B, 2, 3, 1, 1, 128)
+    out, lse = run_dense(p)
+    rows = np.array([[b, 0, i] for b in (0, 1, 65535, 65536, B - 1) for i in (0, 1)],
+                    dtype=np.int32)
+    ro, rl = oracle.attention_rows(p.q, p.k, p.v, rows)
+    o = out.float().cpu()
+    l = lse.cpu()
+    go = np.stack([o[b, i, h].numpy() for b, h, i in rows])
+    gl = np.array([float(l[b, h, i]) for b, h, i in rows])
+    compare(go, gl, ro, rl, what="B=70000")
+
+
+def test_invalid_arguments_raise_and_write_nothing():
+    q = torch.randn(1, 16, 4, 64, device=DEV, dtype=torch.bfloat16)
+    with pytest.raises(fa.FAError) as e:
+        fa.fa_fwd(q, q, q)
+    assert e.value.name == "FA_ERR_UNSUPPORTED"
+    q = torch.randn(1, 16, 4, 128, device=DEV, dtype=torch.bfloat16)
+    k = torch.randn(1, 16, 3, 128, device=DEV, dtype=torch.bfloat16)
+    out = torch.full_like(q, 7.0)
+    with pytest.raises(fa.FAError):
+        fa.fa_fwd(q, k, k, out=out)
+    torch.cuda.synchronize()
+    assert (out == 7.0).all()
