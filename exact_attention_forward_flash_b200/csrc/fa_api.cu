@@ -144,6 +144,9 @@ fa_status validate(const Common &c) {
     if (c.R <= 0 || c.R % 128 != 0)
       return fail(FA_ERR_INVALID, "rel_extent (%d) must be a positive multiple of 128", c.R);
     if (!aligned16(c.rel_bias)) return fail(FA_ERR_INVALID, "rel_bias must be 16-byte aligned");
+    const long long tqb = c.varlen ? c.total_q : (long long)c.B * c.Sq;
+    if (tqb * c.Hq * (long long)c.R / 8 >= (1LL << 32))
+      return fail(FA_ERR_UNSUPPORTED, "rel_bias larger than 64 GiB");
   }
   if (!std::isfinite(c.scale)) return fail(FA_ERR_INVALID, "softmax_scale must be finite");
   const long long tq = c.varlen ? c.total_q : (long long)c.B * c.Sq;
@@ -164,6 +167,7 @@ fa_status validate(const Common &c) {
 }
 
 // Query heads packed per tile: all heads of a K/V group when that divides 128.
+// (a divisor of 128, hence a power of two)
 int pack_factor(int G) { return (G >= 1 && G <= 128 && 128 % G == 0) ? G : 1; }
 
 fa_status fill_params(const Common &c, FwdParams &p, int nq, int bn, int num_splits,
@@ -197,6 +201,8 @@ fa_status fill_params(const Common &c, FwdParams &p, int nq, int bn, int num_spl
   p.Hkv = c.Hkv;
   p.G = G;
   p.P = P;
+  p.lgP = 0;
+  while ((1 << p.lgP) < P) ++p.lgP;
   p.n_groups = c.Hq / P;
   p.total_q = (int)tq;
   const int max_q = c.varlen ? c.max_q : c.Sq;
@@ -205,6 +211,7 @@ fa_status fill_params(const Common &c, FwdParams &p, int nq, int bn, int num_spl
   p.num_splits = num_splits;
   p.split_keys = split_keys;
   p.causal = c.causal ? 1 : 0;
+  p.m_major = c.causal ? 1 : 0;
   p.lse_dense = c.varlen ? 0 : 1;
   const long long units = (long long)c.B * p.n_groups * p.n_mblk * num_splits;
   if (units > 0x7fffffffLL) return fail(FA_ERR_UNSUPPORTED, "too many work units");

@@ -57,12 +57,13 @@ struct FwdParams {
   const int *seqused_k;          // nullptr or [B]
   const uint16_t *rel_bias;      // nullptr or [tok, Hq, R]
   int R;
-  int B, Sq, Sk, Hq, Hkv, G, P, n_groups;
+  int B, Sq, Sk, Hq, Hkv, G, P, lgP, n_groups;
   int total_q;
   int n_mblk;        // CTA tiles per (batch, head group, split)
   int num_splits;
   int split_keys;    // keys per split (multiple of BN); >= any k_len when 1 split
   int causal;
+  int m_major;       // unit order: 1 = largest tile index first over all heads
   int lse_dense;     // 1: lse [B, Hq, Sq]; 0: lse [Hq, total_q]
   int num_units;
   float scale_log2;  // softmax_scale * log2(e)
@@ -81,15 +82,31 @@ struct Unit {
   unsigned active;   // bit t: tile t holds at least one valid row
 };
 
+// Unit u -> (batch, head group, tile index, split).  Causal problems are
+// enumerated tile-index-major from the last (heaviest) tile down, so that the
+// units come roughly sorted by decreasing work across all sequences and
+// heads; other problems keep all tiles of one (batch, head group) together so
+// that concurrently running CTAs share that head's K/V in L2.
 template <int NQ, int BN>
 __device__ __forceinline__ bool decode_unit(const FwdParams &p, int u, Unit &U) {
-  int mblk_rev = u % p.n_mblk;
-  int rest = u / p.n_mblk;
-  U.split = rest % p.num_splits;
-  rest /= p.num_splits;
-  const int grp = rest % p.n_groups;
-  U.b = rest / p.n_groups;
-  const int mblk = p.n_mblk - 1 - mblk_rev;  // heaviest causal tiles first
+  int mblk, grp;
+  if (p.m_major) {
+    const int per_m = p.B * p.n_groups * p.num_splits;
+    const int m_rev = u / per_m;
+    int rest = u - m_rev * per_m;
+    U.split = rest % p.num_splits;
+    rest /= p.num_splits;
+    grp = rest % p.n_groups;
+    U.b = rest / p.n_groups;
+    mblk = p.n_mblk - 1 - m_rev;
+  } else {
+    mblk = u % p.n_mblk;
+    int rest = u / p.n_mblk;
+    U.split = rest % p.num_splits;
+    rest /= p.num_splits;
+    grp = rest % p.n_groups;
+    U.b = rest / p.n_groups;
+  }
   U.hq0 = grp * p.P;
   U.hk = U.hq0 / p.G;
   if (p.cu_q != nullptr) {
@@ -121,6 +138,15 @@ __device__ __forceinline__ bool decode_unit(const FwdParams &p, int u, Unit &U) 
   U.kv_hi = (int)max(hi, lo);
   U.nb = (U.kv_hi - U.kv_lo + BN - 1) / BN;
   return true;
+}
+
+// The k-th unit of this CTA in a static schedule of whole rounds of gridDim.x
+// units whose direction alternates (a "snake"): with units sorted by
+// decreasing work, each CTA's heavy and light picks even out.
+__device__ __forceinline__ int unit_of(int k) {
+  const int G = static_cast<int>(gridDim.x);
+  const int c = static_cast<int>(blockIdx.x);
+  return k * G + ((k & 1) ? (G - 1 - c) : c);
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout: start
@@ -158,7 +184,12 @@ struct FwdCfg {
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + NQ * kQTile;
   static constexpr int kVOff = kKOff + KST * kKVTile;
-  static constexpr int kBarOff = kVOff + VST * kKVTile;
+  // relative-bias staging: one 32-row x 5 x 16-byte buffer per softmax warp,
+  // when shared memory allows (otherwise each thread reads its own row)
+  static constexpr int kBiasWarpBytes = 32 * 3 * 16;
+  static constexpr int kBiasOff = kVOff + VST * kKVTile;
+  static constexpr bool kBiasSmem = kBiasOff + NQ * 4 * kBiasWarpBytes + 1024 + 256 <= 232448;
+  static constexpr int kBarOff = kBiasOff + (kBiasSmem ? NQ * 4 * kBiasWarpBytes : 0);
   // barrier indices
   static constexpr int bQFull = 0, bQEmpty = NQ, bKFull = 2 * NQ, bKEmpty = bKFull + KST,
                        bVFull = bKEmpty + KST, bVEmpty = bVFull + VST, bSFull = bVEmpty + VST,
@@ -167,6 +198,12 @@ struct FwdCfg {
   static constexpr int kSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kSlotOff + 16 + 1024;  // + alignment slack
   static constexpr int kThreads = 128 * (1 + NQ);
+  // registers: with two softmax warpgroups the launch budget (65536 / 384
+  // threads = 168 each) is re-split so that the softmax warps hold a whole
+  // score row plus the bias staging without spilling.
+  static constexpr bool kSplitRegs = NQ == 2;
+  static constexpr uint32_t kRegsCtl = 104, kRegsSoftmax = 200;
+  static_assert(!kSplitRegs || 128 * kRegsCtl + 256 * kRegsSoftmax <= 384 * 168, "register split");
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kOColBase = NQ * NS * BN;
   static_assert(kOColBase + NQ * D <= 512, "tensor memory budget");
@@ -187,9 +224,10 @@ __device__ __forceinline__ void role_producer(const FwdParams &p, uint32_t sb) {
   for (int t = 0; t < C::NQ; ++t) q_cnt[t] = 0;
   uint32_t k_cnt = 0, v_cnt = 0;
   bool ok = true;
-  for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+  for (int k = 0; k * (int)gridDim.x < p.num_units && ok; ++k) {
+    const int u = unit_of(k);
     Unit U;
-    if (!decode_unit<C::NQ, C::BN>(p, u, U) || U.nb == 0) continue;
+    if (u >= p.num_units || !decode_unit<C::NQ, C::BN>(p, u, U) || U.nb == 0) continue;
 #pragma unroll
     for (int t = 0; t < C::NQ; ++t) {
       if (!(U.active >> t & 1u)) continue;
@@ -286,9 +324,10 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
     tc_commit(bar(C::bOFull + t * C::NS + g % C::NS));
   };
 
-  for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+  for (int k = 0; k * (int)gridDim.x < p.num_units && ok; ++k) {
+    const int u = unit_of(k);
     Unit U;
-    if (!decode_unit<C::NQ, C::BN>(p, u, U) || U.nb == 0) continue;
+    if (u >= p.num_units || !decode_unit<C::NQ, C::BN>(p, u, U) || U.nb == 0) continue;
     const int nb = U.nb;
     const int last_t = (U.active >> 1 & 1u) && C::NQ > 1 ? 1 : 0;
     uint32_t sbase[C::NQ];
@@ -378,34 +417,141 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
 // ---------------------------------------------------------------------------
 // softmax / correction / epilogue warpgroup (one per Q tile)
 // ---------------------------------------------------------------------------
+// Relative bias of one 16-column chunk for the 32 rows of one warp.
+//
+// Row i of the tile needs, for columns c = 16*cc + e (e = 0..15), the bias at
+// distance d = base - c with base = i + (k_len - q_len) - j0.  Those 16 values
+// lie inside the 16-byte-aligned run of 24 values that starts at
+//     a = (base - 16*cc - 15) & ~7,
+// i.e. three 16-byte pieces.  The warp fetches the 32 rows x 3 pieces with
+// lane-contiguous 16-byte loads (piece idx = lane + 32*k belongs to row idx/3;
+// consecutive lanes read consecutive pieces of a row, so a load touches few
+// cache lines), stages them in a per-warp shared buffer, and every thread then
+// reads its own row's three pieces back.  Pieces are either wholly inside
+// [0, rel_extent) or wholly outside (both ends are multiples of 8); those
+// outside are zero.
+constexpr int kBiasPieces = 3;
+
+struct BiasFetch {
+  int i[kBiasPieces];         // query position of the row behind each piece, or a sentinel
+  uint32_t off[kBiasPieces];  // offset of that row's bias vector, in 16-byte units
+};
+
+template <class C>
+__device__ __forceinline__ void bias_fetch(const FwdParams &p, const BiasFetch &f, int delta,
+                                           int j0, int cc, uint4 (&pf)[kBiasPieces]) {
+  const uint4 *base = reinterpret_cast<const uint4 *>(p.rel_bias);
+#pragma unroll
+  for (int k = 0; k < kBiasPieces; ++k) {
+    const int pc = (int)((threadIdx.x & 31u) + 32u * k) % kBiasPieces;  // piece within the row
+    const int d0 = ((f.i[k] + delta - j0 - 15 - 16 * cc) & ~7) + 8 * pc;
+    const bool in = d0 >= 0 && d0 + 8 <= p.R;
+    pf[k] = in ? ldg_v4(base + f.off[k] + (d0 >> 3)) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// Add the staged chunk to the thread's scores s[16*CC .. 16*CC + 15].
+template <class C, int CC>
+__device__ __forceinline__ void bias_apply(uint32_t buf, int lane, int sh, float inv_scale,
+                                           float (&s)[C::BN]) {
+  uint32_t w[4 * kBiasPieces];
+#pragma unroll
+  for (int k = 0; k < kBiasPieces; ++k) {
+    const uint4 v = lds_v4(buf + (lane * kBiasPieces + k) * 16);
+    w[4 * k] = v.x;
+    w[4 * k + 1] = v.y;
+    w[4 * k + 2] = v.z;
+    w[4 * k + 3] = v.w;
+  }
+  // align the run so that element 0 is the value at d = base - 16*CC - 15:
+  // shift by sh = 0..7 elements = (sh >> 1) words, then (sh & 1) half words
+  const int sw = sh >> 1;
+#pragma unroll
+  for (int k = 0; k < 10; ++k) w[k] = (sw & 2) ? w[k + 2] : w[k];
+#pragma unroll
+  for (int k = 0; k < 9; ++k) w[k] = (sw & 1) ? w[k + 1] : w[k];
+  const uint32_t sel = (sh & 1) ? 0x5432u : 0x3210u;
+#pragma unroll
+  for (int e2 = 0; e2 < 8; ++e2) {
+    const uint32_t o = __byte_perm(w[e2], w[e2 + 1], sel);
+    // aligned element q = 2*e2 (low half) is column 15 - q of the chunk
+    s[16 * CC + 15 - 2 * e2] = fmaf(lo_f<C::HALF>(o), inv_scale, s[16 * CC + 15 - 2 * e2]);
+    s[16 * CC + 14 - 2 * e2] = fmaf(hi_f<C::HALF>(o), inv_scale, s[16 * CC + 14 - 2 * e2]);
+  }
+}
+
+// Stage and apply chunks CC.. of the bias; the fetch of chunk CC+1 is issued
+// before chunk CC is applied so that its latency overlaps the arithmetic.
+template <class C, int CC>
+__device__ __forceinline__ void bias_chunks(const FwdParams &p, const BiasFetch &bf, int delta,
+                                            int j0, uint32_t buf, int lane, int sh,
+                                            uint4 (&pf)[kBiasPieces], float (&s)[C::BN]) {
+  if constexpr (CC < C::BN / 16) {
+    __syncwarp();
+#pragma unroll
+    for (int kk = 0; kk < kBiasPieces; ++kk) sts_v4(buf + (lane + 32 * kk) * 16, pf[kk]);
+    __syncwarp();
+    if constexpr (CC + 1 < C::BN / 16) bias_fetch<C>(p, bf, delta, j0, CC + 1, pf);
+    bias_apply<C, CC>(buf, lane, sh, p.inv_scale, s);
+    bias_chunks<C, CC + 1>(p, bf, delta, j0, buf, lane, sh, pf, s);
+  }
+}
+
 template <class C>
 __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, uint32_t tmem,
                                              int t) {
   auto bar = [&](int i) { return sb + C::kBarOff + 8u * i; };
   constexpr int BN = C::BN, D = C::D, NS = C::NS;
   const int tid = static_cast<int>(threadIdx.x) - 128 * (t + 1);  // tile row == TMEM lane
+  const int lane = tid & 31;
   const uint32_t lane_addr = static_cast<uint32_t>(tid & ~31) << 16;
+  const uint32_t bias_buf = sb + C::kBiasOff + (t * 4 + (tid >> 5)) * C::kBiasWarpBytes;
   const float sl2 = p.scale_log2;
   uint32_t s_cnt = 0;
   bool ok = true;
 
-  for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+  for (int k = 0; k * (int)gridDim.x < p.num_units && ok; ++k) {
+    const int u = unit_of(k);
     Unit U;
-    if (!decode_unit<C::NQ, BN>(p, u, U) || !(U.active >> t & 1u)) continue;
+    if (u >= p.num_units || !decode_unit<C::NQ, BN>(p, u, U) || !(U.active >> t & 1u)) continue;
     const int row = U.row0 + t * kBM + tid;
-    const int i = row / p.P;
-    const int h = U.hq0 + row % p.P;
+    const int i = row >> p.lgP;
+    const int h = U.hq0 + (row & (p.P - 1));
     const bool valid = i < U.q_len;
     const bool warp_on = __any_sync(0xffffffffu, valid);
     const int lim = p.causal ? min(U.kv_hi, i + U.delta + 1) : U.kv_hi;  // keys j < lim
+    const bool has_bias = p.rel_bias != nullptr;
     const uint16_t *brow = nullptr;
-    if (p.rel_bias != nullptr && valid)
-      brow = p.rel_bias + ((size_t)(U.q_start + i) * p.Hq + h) * p.R;
+    if (has_bias && valid) brow = p.rel_bias + ((size_t)(U.q_start + i) * p.Hq + h) * p.R;
+    BiasFetch bf;
+    if constexpr (C::kBiasSmem) {
+      if (has_bias) {
+#pragma unroll
+        for (int kk = 0; kk < kBiasPieces; ++kk) {
+          const int idx = lane + 32 * kk;
+          const int rr = U.row0 + t * kBM + (tid & ~31) + idx / kBiasPieces;
+          const int ii = rr >> p.lgP;
+          const int hh = U.hq0 + (rr & (p.P - 1));
+          const bool v = ii < U.q_len;
+          bf.i[kk] = v ? ii : -(1 << 30);
+          bf.off[kk] = v ? (uint32_t)((((size_t)(U.q_start + ii) * p.Hq + hh) * p.R) >> 3) : 0u;
+        }
+      }
+    }
 
     float m_ref = -INFINITY, l = 0.f;
     for (int n = 0; n < U.nb; ++n) {
       const uint32_t g = s_cnt + n;
       const uint32_t buf = g % NS;
+      const int j0 = U.kv_lo + n * BN;
+      const int base = i + U.delta - j0;  // distance of column 0
+      // does any row of this warp meet the bias band in this KV tile?
+      const bool bias_blk = __any_sync(0xffffffffu, has_bias && valid && base >= 0 &&
+                                                        base - (BN - 1) < p.R);
+      uint4 pf[kBiasPieces];
+      if constexpr (C::kBiasSmem) {
+        if (bias_blk) bias_fetch<C>(p, bf, U.delta, j0, 0, pf);  // in flight during the wait
+      }
       ok = __all_sync(0xffffffffu,
                       mbar_wait(bar(C::bSFull + t * NS + buf), (g / NS) & 1u, &g_fa_error,
                                 p.timeout_ns));
@@ -422,11 +568,13 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
           for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(r[e]);
         }
         tmem_wait_ld();
-        const int j0 = U.kv_lo + n * BN;
         // relative bias: column c sits at distance d = base - c
-        if (brow != nullptr) {
-          const int base = i + U.delta - j0;
-          if (base >= 0 && base - (BN - 1) < p.R) {
+        if constexpr (C::kBiasSmem) {
+          if (bias_blk) {
+            bias_chunks<C, 0>(p, bf, U.delta, j0, bias_buf, lane, (base - 15) & 7, pf, s);
+          }
+        } else {
+          if (brow != nullptr && base >= 0 && base - (BN - 1) < p.R) {
 #pragma unroll
             for (int c = 0; c < BN; ++c) {
               const int d = base - c;
@@ -591,11 +739,15 @@ __global__ void __launch_bounds__(C::kThreads, 1) fa_fwd_kernel(const __grid_con
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + C::kSlotOff);
 
-  if (warp == 0) {
-    if (lane == 0) role_producer<C>(p, sb);
-  } else if (warp == 1) {
-    if (lane == 0) role_mma<C>(p, sb, tmem);
-  } else if (warp >= 4) {
+  if (warp < 4) {
+    if constexpr (C::kSplitRegs) regs_lower<C::kRegsCtl>();
+    if (warp == 0) {
+      if (lane == 0) role_producer<C>(p, sb);
+    } else if (warp == 1) {
+      if (lane == 0) role_mma<C>(p, sb, tmem);
+    }
+  } else {
+    if constexpr (C::kSplitRegs) regs_raise<C::kRegsSoftmax>();
     role_softmax<C>(p, sb, tmem, warp / 4 - 1);
   }
   __syncwarp();

@@ -9,6 +9,7 @@
 
 #include <cstdint>
 #include <cuda.h>
+#include <cuda_fp16.h>
 
 namespace fab {
 
@@ -217,6 +218,43 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 }
 
 // ---------------------------------------------------------------------------
+// register budget hand-over between warpgroups (all warps of a warpgroup
+// execute the same instruction)
+// ---------------------------------------------------------------------------
+template <uint32_t N>
+__device__ __forceinline__ void regs_raise() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_lower() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// 16-byte read-only global load that bypasses L1 allocation policy hints.
+__device__ __forceinline__ uint4 ldg_v4(const void *p) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void sts_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"(addr)
+               : "memory");
+  return r;
+}
+
+// ---------------------------------------------------------------------------
 // arithmetic helpers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -241,6 +279,22 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   else
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// The low / high 16-bit element of a word, widened to float.
+template <bool kHalf>
+__device__ __forceinline__ float lo_f(uint32_t w) {
+  if constexpr (kHalf)
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xffffu)));
+  else
+    return __uint_as_float(w << 16);
+}
+template <bool kHalf>
+__device__ __forceinline__ float hi_f(uint32_t w) {
+  if constexpr (kHalf)
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
+  else
+    return __uint_as_float(w & 0xffff0000u);
 }
 
 template <bool kHalf>

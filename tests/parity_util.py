@@ -58,7 +58,7 @@ def lse_rows(lse_dense_bhs, rows):
     return np.array([l[b, h, i] for b, h, i in rows])
 
 
-def compare_relative(out, ref_o, *, ulps=2.0, floor=2e-3, what=""):
+def compare_relative(out, ref_o, *, ulps=2.0, floor=1e-2, what=""):
     """Stress inputs (sharp softmax, large bias or offset values): |O| reaches
     several units, where one bf16 ulp alone exceeds the absolute gate.  Gate
     each element at `ulps` bf16 ulps of the reference plus a small floor."""

@@ -289,8 +289,10 @@ def test_stress_peaked_and_offset_values():
 def test_many_batches_beyond_grid_y_limit():
     # batch x heads well past 65535 (the grid-dimension limit a kernel that
     # put them in gridDim.y would hit)
+    # 40 keys keep |O| small, so that the output's bf16 rounding stays below
+    # the mean-abs gate
     B = 70000
-    p = fa_inputs.random_dense(35, B, 2, 3, 1, 1, 128)
+    p = fa_inputs.random_dense(35, B, 2, 40, 1, 1, 128)
     out, lse = run_dense(p)
     rows = np.array([[b, 0, i] for b in (0, 1, 65535, 65536, B - 1) for i in (0, 1)],
                     dtype=np.int32)
