@@ -433,27 +433,59 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
 constexpr int kBiasPieces = 3;
 
 struct BiasFetch {
-  int i[kBiasPieces];         // query position of the row behind each piece, or a sentinel
+  int b0[kBiasPieces];        // distance of column 0 of the unit's first KV tile for the
+                              // row behind each piece (i + k_len - q_len - kv_lo), or a
+                              // sentinel far below zero for rows past the sequence
   uint32_t off[kBiasPieces];  // offset of that row's bias vector, in 16-byte units
 };
 
+// The bias loads of a tile go out in two batches of NC/2 chunks (one per
+// 64-column half): the first before the thread waits for the tile's scores
+// (their latency hides behind that wait), the second once the first half has
+// taken its bias.  A chunk that no row of the warp meets is neither fetched
+// nor staged.
 template <class C>
-__device__ __forceinline__ void bias_fetch(const FwdParams &p, const BiasFetch &f, int delta,
-                                           int j0, int cc, uint4 (&pf)[kBiasPieces]) {
-  const uint4 *base = reinterpret_cast<const uint4 *>(p.rel_bias);
+__device__ __forceinline__ unsigned bias_need(const FwdParams &p, int base, bool row_on) {
+  unsigned need = 0;  // warp-uniform: chunks that some row of the warp meets
+#pragma unroll
+  for (int cc = 0; cc < C::BN / 16; ++cc) {
+    const bool nd = row_on && base - 16 * cc >= 0 && base - 16 * cc - 15 < p.R;
+    need |= (__any_sync(0xffffffffu, nd) ? 1u : 0u) << cc;
+  }
+  return need;
+}
+
+// Issue the loads of chunks [C0, C0 + H) into pf.
+template <class C, int C0>
+__device__ __forceinline__ void bias_load(const FwdParams &p, const BiasFetch &bf, int jrel,
+                                          int lane, unsigned need,
+                                          uint4 (&pf)[4][kBiasPieces]) {
+  constexpr int H = 4;  // chunks of one 64-column half
 #pragma unroll
   for (int k = 0; k < kBiasPieces; ++k) {
-    const int pc = (int)((threadIdx.x & 31u) + 32u * k) % kBiasPieces;  // piece within the row
-    const int d0 = ((f.i[k] + delta - j0 - 15 - 16 * cc) & ~7) + 8 * pc;
-    const bool in = d0 >= 0 && d0 + 8 <= p.R;
-    pf[k] = in ? ldg_v4(base + f.off[k] + (d0 >> 3)) : make_uint4(0u, 0u, 0u, 0u);
+    const int pc = (lane + 32 * k) % kBiasPieces;  // piece index within the row
+    const int d00 = ((bf.b0[k] - jrel - 15) & ~7) + 8 * pc;
+    const uint4 *rp = reinterpret_cast<const uint4 *>(p.rel_bias) + bf.off[k];
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
+      const int cc = C0 + h;
+      const int d0 = d00 - 16 * cc;  // chunk cc sits 16*cc elements lower
+      const bool in = (need >> cc & 1u) && d0 >= 0 && d0 + 8 <= p.R;
+      pf[h][k] = in ? ldg_v4(rp + (d0 >> 3)) : make_uint4(0u, 0u, 0u, 0u);
+    }
   }
 }
 
-// Add the staged chunk to the thread's scores s[16*CC .. 16*CC + 15].
-template <class C, int CC>
-__device__ __forceinline__ void bias_apply(uint32_t buf, int lane, int sh, float inv_scale,
-                                           float (&s)[C::BN]) {
+// Transpose chunk pieces through the warp's buffer and return this row's 16
+// bias values as 16-bit pairs in column order (w2[k]: columns 2k, 2k+1).
+template <class C>
+__device__ __forceinline__ void bias_chunk(uint32_t buf, int lane, int sh,
+                                           const uint4 (&pieces)[kBiasPieces],
+                                           uint32_t (&w2)[8]) {
+  __syncwarp();
+#pragma unroll
+  for (int k = 0; k < kBiasPieces; ++k) sts_v4(buf + (lane + 32 * k) * 16, pieces[k]);
+  __syncwarp();
   uint32_t w[4 * kBiasPieces];
 #pragma unroll
   for (int k = 0; k < kBiasPieces; ++k) {
@@ -463,38 +495,17 @@ __device__ __forceinline__ void bias_apply(uint32_t buf, int lane, int sh, float
     w[4 * k + 2] = v.z;
     w[4 * k + 3] = v.w;
   }
-  // align the run so that element 0 is the value at d = base - 16*CC - 15:
-  // shift by sh = 0..7 elements = (sh >> 1) words, then (sh & 1) half words
+  // element q of the aligned run (q = 0..15) is the value at distance
+  // base - 16*cc - 15 + q, i.e. column 15 - q of the chunk
   const int sw = sh >> 1;
 #pragma unroll
   for (int k = 0; k < 10; ++k) w[k] = (sw & 2) ? w[k + 2] : w[k];
 #pragma unroll
   for (int k = 0; k < 9; ++k) w[k] = (sw & 1) ? w[k + 1] : w[k];
-  const uint32_t sel = (sh & 1) ? 0x5432u : 0x3210u;
+  // pick two consecutive aligned elements, swapped into column order
+  const uint32_t sel = (sh & 1) ? 0x3254u : 0x1032u;
 #pragma unroll
-  for (int e2 = 0; e2 < 8; ++e2) {
-    const uint32_t o = __byte_perm(w[e2], w[e2 + 1], sel);
-    // aligned element q = 2*e2 (low half) is column 15 - q of the chunk
-    s[16 * CC + 15 - 2 * e2] = fmaf(lo_f<C::HALF>(o), inv_scale, s[16 * CC + 15 - 2 * e2]);
-    s[16 * CC + 14 - 2 * e2] = fmaf(hi_f<C::HALF>(o), inv_scale, s[16 * CC + 14 - 2 * e2]);
-  }
-}
-
-// Stage and apply chunks CC.. of the bias; the fetch of chunk CC+1 is issued
-// before chunk CC is applied so that its latency overlaps the arithmetic.
-template <class C, int CC>
-__device__ __forceinline__ void bias_chunks(const FwdParams &p, const BiasFetch &bf, int delta,
-                                            int j0, uint32_t buf, int lane, int sh,
-                                            uint4 (&pf)[kBiasPieces], float (&s)[C::BN]) {
-  if constexpr (CC < C::BN / 16) {
-    __syncwarp();
-#pragma unroll
-    for (int kk = 0; kk < kBiasPieces; ++kk) sts_v4(buf + (lane + 32 * kk) * 16, pf[kk]);
-    __syncwarp();
-    if constexpr (CC + 1 < C::BN / 16) bias_fetch<C>(p, bf, delta, j0, CC + 1, pf);
-    bias_apply<C, CC>(buf, lane, sh, p.inv_scale, s);
-    bias_chunks<C, CC + 1>(p, bf, delta, j0, buf, lane, sh, pf, s);
-  }
+  for (int e2 = 0; e2 < 8; ++e2) w2[7 - e2] = __byte_perm(w[e2], w[e2 + 1], sel);
 }
 
 template <class C>
@@ -519,10 +530,27 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
     const int h = U.hq0 + (row & (p.P - 1));
     const bool valid = i < U.q_len;
     const bool warp_on = __any_sync(0xffffffffu, valid);
-    const int lim = p.causal ? min(U.kv_hi, i + U.delta + 1) : U.kv_hi;  // keys j < lim
+    const int nb = U.nb;
+    // per-row constants relative to the unit's first key kv_lo, so that the
+    // unit record can die before the KV loop
+    const int lim_rel = (p.causal ? min(U.kv_hi, i + U.delta + 1) : U.kv_hi) - U.kv_lo;
+    const int base0 = i + U.delta - U.kv_lo;  // distance of column 0 of tile 0
+    const size_t orow = (size_t)(U.q_start + i) * p.Hq + h;  // packed (token, head) row
+    void *out_row;
+    float *lse_ptr;
+    if constexpr (C::PARTIAL) {
+      const size_t prow = (size_t)U.split * p.total_q * p.Hq + orow;
+      out_row = p.o_part + prow * D;
+      lse_ptr = p.lse_part + prow;
+    } else {
+      out_row = reinterpret_cast<uint16_t *>(p.out) + orow * D;
+      lse_ptr = p.lse == nullptr ? nullptr
+                : p.lse + (p.lse_dense ? ((size_t)U.b * p.Hq + h) * p.Sq + i
+                                       : (size_t)h * p.total_q + U.q_start + i);
+    }
     const bool has_bias = p.rel_bias != nullptr;
     const uint16_t *brow = nullptr;
-    if (has_bias && valid) brow = p.rel_bias + ((size_t)(U.q_start + i) * p.Hq + h) * p.R;
+    if (has_bias && valid) brow = p.rel_bias + orow * p.R;
     BiasFetch bf;
     if constexpr (C::kBiasSmem) {
       if (has_bias) {
@@ -533,112 +561,237 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
           const int ii = rr >> p.lgP;
           const int hh = U.hq0 + (rr & (p.P - 1));
           const bool v = ii < U.q_len;
-          bf.i[kk] = v ? ii : -(1 << 30);
+          bf.b0[kk] = v ? ii + U.delta - U.kv_lo : -(1 << 30);
           bf.off[kk] = v ? (uint32_t)((((size_t)(U.q_start + ii) * p.Hq + hh) * p.R) >> 3) : 0u;
         }
       }
     }
 
     float m_ref = -INFINITY, l = 0.f;
-    for (int n = 0; n < U.nb; ++n) {
+    for (int n = 0; n < nb; ++n) {
       const uint32_t g = s_cnt + n;
       const uint32_t buf = g % NS;
-      const int j0 = U.kv_lo + n * BN;
-      const int base = i + U.delta - j0;  // distance of column 0
+      const int jrel = n * BN;
+      const int base = base0 - jrel;  // distance of column 0
       // does any row of this warp meet the bias band in this KV tile?
       const bool bias_blk = __any_sync(0xffffffffu, has_bias && valid && base >= 0 &&
                                                         base - (BN - 1) < p.R);
-      uint4 pf[kBiasPieces];
-      if constexpr (C::kBiasSmem) {
-        if (bias_blk) bias_fetch<C>(p, bf, U.delta, j0, 0, pf);  // in flight during the wait
-      }
-      ok = __all_sync(0xffffffffu,
-                      mbar_wait(bar(C::bSFull + t * NS + buf), (g / NS) & 1u, &g_fa_error,
-                                p.timeout_ns));
-      if (!ok) break;
-      tc_fence_after();
-      if (warp_on) {
-        const uint32_t s_addr = tmem + lane_addr + C::s_col(t, buf);
-        float s[BN];
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(s_addr + 32 * c, r);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(r[e]);
-        }
-        tmem_wait_ld();
-        // relative bias: column c sits at distance d = base - c
-        if constexpr (C::kBiasSmem) {
-          if (bias_blk) {
-            bias_chunks<C, 0>(p, bf, U.delta, j0, bias_buf, lane, (base - 15) & 7, pf, s);
+      const uint32_t s_addr = tmem + lane_addr + C::s_col(t, buf);
+      const int lim_c = lim_rel - jrel;  // columns at or past lim_c are masked
+      auto wait_scores = [&]() -> bool {
+        const bool w = __all_sync(0xffffffffu,
+                                  mbar_wait(bar(C::bSFull + t * NS + buf), (g / NS) & 1u,
+                                            &g_fa_error, p.timeout_ns));
+        tc_fence_after();
+        return w;
+      };
+      // O (and l) rescale by f once the running max has moved; for n > 0
+        // the previous P.V must have completed (guaranteed by the score
+        // barrier when S is single-buffered, waited for otherwise).
+        auto rescale_o = [&](float f) -> bool {
+          if (NS == 2) {
+            const uint32_t gp = g - 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(C::bOFull + t * NS + gp % NS),
+                                                   (gp / NS) & 1u, &g_fa_error, p.timeout_ns)))
+              return false;
+            tc_fence_after();
           }
-        } else {
-          if (brow != nullptr && base >= 0 && base - (BN - 1) < p.R) {
-#pragma unroll
-            for (int c = 0; c < BN; ++c) {
-              const int d = base - c;
-              if (d >= 0 && d < p.R) s[c] += load_elem<C::HALF>(brow + d) * p.inv_scale;
-            }
-          }
-        }
-        // masks: keys at or past `lim` (end of keys / causal diagonal)
-        const int lim_c = lim - j0;
-        if (lim_c < BN) {
-#pragma unroll
-          for (int c = 0; c < BN; ++c)
-            if (c >= lim_c) s[c] = -INFINITY;
-        }
-        float mx = s[0];
-#pragma unroll
-        for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
-        const float m_new = fmaxf(m_ref, mx);
-        if (n == 0) {
-          m_ref = m_new;
-        } else {
-          const bool need = (m_new - m_ref) > p.thr_raw;
-          if (__any_sync(0xffffffffu, need)) {
-            if (NS == 2) {  // the previous P.V must have landed in O
-              const uint32_t gp = g - 1;
-              ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bOFull + t * NS + gp % NS),
-                                                     (gp / NS) & 1u, &g_fa_error, p.timeout_ns));
-              if (!ok) break;
-              tc_fence_after();
-            }
-            const float f = need ? ex2_approx((m_ref - m_new) * sl2) : 1.f;
-            if (need) {
-              l *= f;
-              m_ref = m_new;
-            }
-            const uint32_t o_addr = tmem + lane_addr + C::o_col(t);
+          const uint32_t o_addr = tmem + lane_addr + C::o_col(t);
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t r[32];
-              tmem_ld32(o_addr + 32 * c, r);
-              tmem_wait_ld();
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(o_addr + 32 * c, o);
+            tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
-              tmem_st32(o_addr + 32 * c, r);
-            }
-            tmem_wait_st();
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            tmem_st32(o_addr + 32 * c, o);
           }
-        }
-        const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * sl2;
-        float lsum = 0.f;
+          return true;
+        };
+      // The two kinds of tile take disjoint paths (each with its own wait) so
+      // that their register-resident arrays never meet at a join.
+      if (C::kBiasSmem && bias_blk) {
+        const unsigned need = bias_need<C>(p, base, valid);
+        uint4 pf[4][kBiasPieces];  // bias pieces of one 64-column half
+        bias_load<C, 0>(p, bf, jrel, lane, need, pf);  // in flight during the wait
+        ok = wait_scores();
+        if (!ok) break;
+        if (warp_on) {
+          // Tiles that meet the bias band: 64-column halves, each with its own
+          // running-max update (online softmax at half-tile granularity), so
+          // that the staged bias and the scores fit in registers together.
+          // With conditional rescaling the second half rarely moves the
+          // reference max; when it does, the first half's P (already in tensor
+          // memory) is rescaled along with O and l.
+          const bool staged = true;
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          s[c] = ex2_approx(fmaf(s[c], sl2, -mc));
-          lsum += s[c];
-        }
-        l += lsum;
+        for (int hf = 0; hf < BN / 64; ++hf) {
+          uint32_t r[64];
+          {
+            uint32_t r0[32], r1[32];
+            tmem_ld32(s_addr + 64 * hf, r0);
+            tmem_ld32(s_addr + 64 * hf + 32, r1);
+            tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < BN / 64; ++c) {
-          uint32_t r[32];
+            for (int e = 0; e < 32; ++e) {
+              r[e] = r0[e];
+              r[32 + e] = r1[e];
+            }
+          }
+          if constexpr (C::kBiasSmem) {
+            if (staged) {
+              const int sh = (base - 15) & 7;  // misalignment of the bias run
 #pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = pack2<C::HALF>(s[64 * c + 2 * e], s[64 * c + 2 * e + 1]);
-          tmem_st32(s_addr + 32 * c, r);
+              for (int cc = 0; cc < 4; ++cc) {
+                if (need >> (4 * hf + cc) & 1u) {
+                  uint32_t w2[8];
+                  bias_chunk<C>(bias_buf, lane, sh, pf[cc], w2);
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) {
+                    r[16 * cc + 2 * e] = __float_as_uint(fmaf(
+                        lo_f<C::HALF>(w2[e]), p.inv_scale, __uint_as_float(r[16 * cc + 2 * e])));
+                    r[16 * cc + 2 * e + 1] = __float_as_uint(fmaf(
+                        hi_f<C::HALF>(w2[e]), p.inv_scale, __uint_as_float(r[16 * cc + 2 * e + 1])));
+                  }
+                }
+              }
+              if (hf + 1 < BN / 64) bias_load<C, 4>(p, bf, jrel, lane, need, pf);
+            }
+          } else {
+            // relative bias without shared staging: column c at distance base - c
+            if (brow != nullptr) {
+#pragma unroll
+              for (int e = 0; e < 64; ++e) {
+                const int d = base - (64 * hf + e);
+                if (d >= 0 && d < p.R)
+                  r[e] = __float_as_uint(__uint_as_float(r[e]) +
+                                         load_elem<C::HALF>(brow + d) * p.inv_scale);
+              }
+            }
+          }
+          float mx = -INFINITY;
+#pragma unroll
+          for (int e = 0; e < 64; ++e) {
+            const float x = (64 * hf + e >= lim_c) ? -INFINITY : __uint_as_float(r[e]);
+            r[e] = __float_as_uint(x);
+            mx = fmaxf(mx, x);
+          }
+          // running-max update with conditional rescaling
+          const float m_new = fmaxf(m_ref, mx);
+          if (n == 0 && hf == 0) {
+            m_ref = m_new;
+          } else {
+            const bool need_rs = (m_new - m_ref) > p.thr_raw;
+            if (__any_sync(0xffffffffu, need_rs)) {
+              const float f = need_rs ? ex2_approx((m_ref - m_new) * sl2) : 1.f;
+              if (need_rs) {
+                l *= f;
+                m_ref = m_new;
+              }
+              if (n > 0) {
+                ok = rescale_o(f);
+                if (!ok) break;
+              }
+              if (hf > 0) {  // P of the earlier halves of this tile
+#pragma unroll 1
+                for (int c = 0; c < hf; ++c) {
+                  uint32_t o[32];
+                  tmem_ld32(s_addr + 32 * c, o);
+                  tmem_wait_ld();
+#pragma unroll
+                  for (int e = 0; e < 32; ++e)
+                    o[e] = pack2<C::HALF>(lo_f<C::HALF>(o[e]) * f, hi_f<C::HALF>(o[e]) * f);
+                  tmem_st32(s_addr + 32 * c, o);
+                }
+              }
+              tmem_wait_st();
+            }
+          }
+          const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * sl2;
+          float lsum = 0.f;
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * e]), sl2, -mc));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * e + 1]), sl2, -mc));
+            lsum += p0 + p1;
+            pk[e] = pack2<C::HALF>(p0, p1);
+          }
+          l += lsum;
+          // P half hf -> columns [32 hf, 32 hf + 32): only score columns
+          // already read are overwritten
+          tmem_st32(s_addr + 32 * hf, pk);
         }
-        tmem_wait_st();
+          if (!ok) break;
+          tmem_wait_st();
+        }
+      } else {
+        ok = wait_scores();
+        if (!ok) break;
+        if (warp_on) {
+          // Tiles without bias: the whole row of scores in registers, one
+          // running-max update per tile.
+          float s[BN];
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(s_addr + 32 * c, r);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(r[e]);
+          }
+          tmem_wait_ld();
+          if constexpr (!C::kBiasSmem) {
+            // relative bias without shared staging: column c at distance base - c
+            if (brow != nullptr && base >= 0 && base - (BN - 1) < p.R) {
+#pragma unroll
+              for (int c = 0; c < BN; ++c) {
+                const int d = base - c;
+                if (d >= 0 && d < p.R) s[c] += load_elem<C::HALF>(brow + d) * p.inv_scale;
+              }
+            }
+          }
+          if (lim_c < BN) {
+#pragma unroll
+            for (int c = 0; c < BN; ++c)
+              if (c >= lim_c) s[c] = -INFINITY;
+          }
+          float mx = s[0];
+#pragma unroll
+          for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+          const float m_new = fmaxf(m_ref, mx);
+          if (n == 0) {
+            m_ref = m_new;
+          } else {
+            const bool need_rs = (m_new - m_ref) > p.thr_raw;
+            if (__any_sync(0xffffffffu, need_rs)) {
+              const float f = need_rs ? ex2_approx((m_ref - m_new) * sl2) : 1.f;
+              if (need_rs) {
+                l *= f;
+                m_ref = m_new;
+              }
+              ok = rescale_o(f);
+              if (!ok) break;
+              tmem_wait_st();
+            }
+          }
+          const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * sl2;
+          float lsum = 0.f;
+#pragma unroll
+          for (int c = 0; c < BN; ++c) {
+            s[c] = ex2_approx(fmaf(s[c], sl2, -mc));
+            lsum += s[c];
+          }
+          l += lsum;
+#pragma unroll
+          for (int c = 0; c < BN / 64; ++c) {
+            uint32_t r[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              r[e] = pack2<C::HALF>(s[64 * c + 2 * e], s[64 * c + 2 * e + 1]);
+            tmem_st32(s_addr + 32 * c, r);
+          }
+          tmem_wait_st();
+        }
       }
       tc_fence_before();
       mbar_arrive(bar(C::bPFull + t * NS + buf));
@@ -648,9 +801,8 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
     // epilogue
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
     const float lse_v = l > 0.f ? (m_ref * sl2 + lg2_approx(l)) * 0.69314718055994531f : -INFINITY;
-    const size_t orow = (size_t)(U.q_start + i) * p.Hq + h;  // packed (token, head) row
-    if (U.nb > 0) {
-      const uint32_t gl = s_cnt + U.nb - 1;
+    if (nb > 0) {
+      const uint32_t gl = s_cnt + nb - 1;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bOFull + t * NS + gl % NS), (gl / NS) & 1u,
                                              &g_fa_error, p.timeout_ns));
       if (!ok) break;
@@ -660,7 +812,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
-        if (U.nb > 0) {
+        if (nb > 0) {
           tmem_ld32(tmem + lane_addr + C::o_col(t) + 32 * c, r);
           tmem_wait_ld();
         } else {
@@ -669,7 +821,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
         }
         if (valid) {
           if constexpr (C::PARTIAL) {
-            float *dst = p.o_part + ((size_t)U.split * p.total_q * p.Hq + orow) * D + 32 * c;
+            float *dst = reinterpret_cast<float *>(out_row) + 32 * c;
 #pragma unroll
             for (int e = 0; e < 32; e += 4) {
               float4 w = make_float4(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l,
@@ -678,7 +830,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
               *reinterpret_cast<float4 *>(dst + e) = w;
             }
           } else {
-            uint16_t *dst = reinterpret_cast<uint16_t *>(p.out) + orow * D + 32 * c;
+            uint16_t *dst = reinterpret_cast<uint16_t *>(out_row) + 32 * c;
 #pragma unroll
             for (int e = 0; e < 32; e += 8) {
               uint4 w;
@@ -692,20 +844,12 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
         }
       }
     }
-    if (valid) {
-      if constexpr (C::PARTIAL) {
-        p.lse_part[(size_t)U.split * p.total_q * p.Hq + orow] = lse_v;
-      } else if (p.lse != nullptr) {
-        const size_t li = p.lse_dense ? ((size_t)U.b * p.Hq + h) * p.Sq + i
-                                      : (size_t)h * p.total_q + U.q_start + i;
-        p.lse[li] = lse_v;
-      }
-    }
-    if (U.nb > 0) {
+    if (valid && lse_ptr != nullptr) *lse_ptr = lse_v;
+    if (nb > 0) {
       tc_fence_before();
       mbar_arrive(bar(C::bOEmpty + t));
     }
-    s_cnt += U.nb;
+    s_cnt += nb;
   }
 }
 

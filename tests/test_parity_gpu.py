@@ -257,14 +257,21 @@ def test_empty_batch_is_a_no_op():
     assert out.numel() == 0
 
 
-def test_bias_none_equals_bias_zero_bitwise():
+def test_bias_none_equals_bias_zero():
+    # tiles that meet the bias band take the half-tile softmax path, so a zero
+    # bias need not reproduce the bias-free path bit for bit; both must meet
+    # the oracle's gates and agree closely with each other
     p = fa_inputs.random_dense(32, 1, 300, 300, 4, 4, 128, causal=True)
     g = p.to(DEV)
     o1, l1 = fa.fa_fwd(g.q, g.k, g.v, causal=True)
     zb = torch.zeros((300, 4, 128), dtype=torch.bfloat16, device=DEV)
     o2, l2 = fa.fa_fwd(g.q, g.k, g.v, causal=True, rel_bias=zb)
     torch.cuda.synchronize()
-    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    ro, rl = ref_dense(p)
+    compare(o1, l1, ro, rl, what="no bias")
+    compare(o2, l2, ro, rl, what="zero bias")
+    assert (o1.float() - o2.float()).abs().max().item() <= 8e-3
+    assert (l1 - l2).abs().max().item() <= 1e-5
 
 
 def test_deterministic_run_to_run():
