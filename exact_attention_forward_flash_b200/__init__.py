@@ -71,6 +71,9 @@ def load_library(path: Optional[str] = None):
                                    i32, i32, i32, f32, P, P, i32, i32, P,
                                    ctypes.c_size_t, P]
     lib.fa_fwd_splitkv.restype = i32
+    lib.fa_fwd_splitkv_static.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32,
+                                          i32, i32, i32, f32, P, P, i32, i32, P]
+    lib.fa_fwd_splitkv_static.restype = i32
     lib.fa_check_device_error.argtypes = [ctypes.POINTER(i32), i32]
     lib.fa_check_device_error.restype = i32
     lib.fa_status_string.argtypes = [i32]
@@ -232,6 +235,35 @@ def fa_fwd_splitkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
         D, _dtype(q), int(bool(causal)), float(softmax_scale or 0.0),
         _ptr(seqused_k), _ptr(rel_bias), R, int(ns), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out, lse
+
+
+def fa_fwd_splitkv_static(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
+                          num_splits: int = 0, causal: bool = False,
+                          softmax_scale: Optional[float] = None,
+                          seqused_k: Optional[torch.Tensor] = None,
+                          rel_bias: Optional[torch.Tensor] = None,
+                          out: Optional[torch.Tensor] = None,
+                          lse: Optional[torch.Tensor] = None,
+                          stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Split-KV dense forward whose partials go to the library's own static
+    scratch (no workspace); for callers that must not allocate device memory.
+    Pass ``out`` and ``lse`` to keep this call free of allocations too."""
+    lib = load_library()
+    B, Sq, Hq, D = q.shape
+    _, Sk, Hkv, _ = k.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    _need_cuda(q, k, v, out, lse, seqused_k, rel_bias)
+    _same_dtype(q, k, v, out, rel_bias)
+    _int32(seqused_k, "seqused_k")
+    R = 0 if rel_bias is None else int(rel_bias.shape[-1])
+    _check(lib.fa_fwd_splitkv_static(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq, Sk, Hq, Hkv,
+        D, _dtype(q), int(bool(causal)), float(softmax_scale or 0.0),
+        _ptr(seqused_k), _ptr(rel_bias), R, int(num_splits), _stream(stream)))
     return out, lse
 
 

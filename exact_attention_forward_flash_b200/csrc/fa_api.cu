@@ -385,3 +385,67 @@ fa_status fa_check_device_error(int *code, int clear) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Split-KV forward without any allocation by the caller or the library.
+//
+// The split partials live in one file-scope device array instead of a
+// caller-provided workspace.  Its size is fixed at build time
+// (FA_SPLITKV_STATIC_SCRATCH_BYTES) and it is held by every GPU that loads
+// this library until the process exits.  Host code only sees a stand-in for
+// the array's name, so its device address is looked up once per device (with
+// that device current) by the first call made on that device.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_splitkv_scratch[FA_SPLITKV_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+fa_status splitkv_scratch_address(int dev, void **addr) {
+  static std::mutex mu;
+  static void *cached[kMaxDev] = {nullptr};
+  if (dev < 0 || dev >= kMaxDev) return fail(FA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == nullptr) {
+    void *ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_splitkv_scratch);
+    if (e != cudaSuccess || ptr == nullptr)
+      return fail(FA_ERR_CUDA, "looking up the static split-KV scratch: %s", cudaGetErrorString(e));
+    cached[dev] = ptr;
+  }
+  *addr = cached[dev];
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" fa_status fa_fwd_splitkv_static(const void *q, const void *k, const void *v, void *out,
+                                           float *lse, int B, int Sq, int Sk, int Hq, int Hkv,
+                                           int D, fa_dtype dt, int causal, float softmax_scale,
+                                           const int *seqused_k, const void *rel_bias,
+                                           int rel_extent, int num_splits, void *stream) {
+  g_msg[0] = 0;
+  if (num_splits < 0) return fail(FA_ERR_INVALID, "num_splits must be >= 0");
+  int dev = 0;
+  if ((long long)B * Sq > 0 && Sk > 0) {
+    if (cudaGetDevice(&dev) != cudaSuccess) return fail(FA_ERR_CUDA, "cudaGetDevice failed");
+    // the split count fa_fwd_splitkv will use, and the scratch it needs
+    const int bn = splitkv_bn(D);
+    int ns = num_splits > 0 ? num_splits
+                            : fa_splitkv_default_splits(B, Sq, Sk, Hq, Hkv, D, num_sms(dev));
+    const long long tiles = ((long long)Sk + bn - 1) / bn;
+    if (ns > tiles) ns = (int)tiles;
+    if (ns < 1) ns = 1;
+    const size_t need = fa_splitkv_workspace_bytes(B, Sq, Hq, D, ns);
+    if (need > (size_t)FA_SPLITKV_STATIC_SCRATCH_BYTES)
+      return fail(FA_ERR_WORKSPACE,
+                  "split-KV partials need %zu bytes, more than the %zu-byte static scratch "
+                  "(use fa_fwd_splitkv with a workspace, or fewer splits)",
+                  need, (size_t)FA_SPLITKV_STATIC_SCRATCH_BYTES);
+  }
+  void *scratch = nullptr;
+  fa_status s = splitkv_scratch_address(dev, &scratch);
+  if (s != FA_OK) return s;
+  return fa_fwd_splitkv(q, k, v, out, lse, B, Sq, Sk, Hq, Hkv, D, dt, causal, softmax_scale,
+                        seqused_k, rel_bias, rel_extent, num_splits, scratch,
+                        (size_t)FA_SPLITKV_STATIC_SCRATCH_BYTES, stream);
+}

@@ -129,6 +129,40 @@ fa_status fa_fwd_splitkv(const void *q, const void *k, const void *v, void *out,
                          size_t workspace_bytes, void *stream);
 
 /*
+ * Split-KV forward that allocates nothing: no workspace argument, and no
+ * device allocation inside the library.  The pages have no counterpart to
+ * this entry point; it exists for callers that cannot call cudaMalloc at all
+ * and so cannot provide fa_fwd_splitkv's workspace: code that runs where the
+ * device allocator belongs to someone else (a host framework's caching
+ * allocator or a memory pool sized once at start-up, which the caller must
+ * not bypass), or code under a rule of no allocation after initialisation
+ * (fixed-latency serving loops, where a cudaMalloc can synchronise the device
+ * and stall every stream).
+ *
+ * The split partials go to a scratch array inside the library of
+ * FA_SPLITKV_STATIC_SCRATCH_BYTES bytes, which every GPU that loads the
+ * library holds until the process exits.  Arguments are those of
+ * fa_fwd_splitkv without the workspace; a problem whose partials
+ * (fa_splitkv_workspace_bytes for the split count used) exceed the scratch is
+ * rejected with FA_ERR_WORKSPACE before anything is enqueued.
+ *
+ * The first call on each device looks up the scratch's device address (with
+ * that device current) and caches it; make that first call before any stream
+ * capture.  All calls share the one array and it keeps the last call's
+ * contents; each call writes every partial it reads, so nothing has to start
+ * at zero.  Calls whose kernels overlap on the GPU (different streams without
+ * ordering between them, or several host threads) race on the array and give
+ * wrong results: order them.
+ */
+#define FA_SPLITKV_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+fa_status fa_fwd_splitkv_static(const void *q, const void *k, const void *v,
+                                void *out, float *lse, int B, int Sq, int Sk,
+                                int Hq, int Hkv, int D, fa_dtype dt,
+                                int causal, float softmax_scale,
+                                const int *seqused_k, const void *rel_bias,
+                                int rel_extent, int num_splits, void *stream);
+
+/*
  * Device-side watchdog.  Every wait inside the kernels is bounded; a kernel
  * that gives up records a code in a device word and returns without
  * trapping.  This call synchronises the current device, copies that word to
