@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--splits", type=int, default=0, help="split-KV count (0 = auto)")
+    ap.add_argument("--decode-sk", type=int, default=131072,
+                    help="keys of the decode workload (smaller values for profiling)")
     return ap.parse_args()
 
 
@@ -166,10 +168,13 @@ class ClockSampler:
 BIG = {"video_dit_20480", "decode_splitkv"}
 
 
+DECODE_SK = 131072
+
+
 def build_problem(name: str, device):
     import fa_inputs
     if name in BIG:
-        return fa_inputs.make(name, device=device)
+        return fa_inputs.make(name, device=device, decode_sk=DECODE_SK)
     return fa_inputs.make(name).to(device)
 
 
@@ -319,6 +324,8 @@ def time_oracle(p_cpu, target_s: float):
 # ---------------------------------------------------------------------------
 def main():
     a = parse()
+    global DECODE_SK
+    DECODE_SK = a.decode_sk
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

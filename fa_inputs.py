@@ -142,13 +142,14 @@ class Problem:
                        dict(self.meta))
 
 
-def make(name: str, dtype=torch.bfloat16, device="cpu") -> Problem:
+def make(name: str, dtype=torch.bfloat16, device="cpu", decode_sk: int = 131072) -> Problem:
     """Build one named workload with its fixed seed.
 
     With ``device`` other than the CPU the values are drawn there by that
     device's seeded generator (another stream of numbers than the CPU
     generator's, same distributions and shapes): the benchmark uses this for
-    the multi-GB workloads; parity tests draw on the CPU."""
+    the multi-GB workloads; parity tests draw on the CPU.  ``decode_sk``
+    shortens the decode workload's keys (for profiling a smaller case)."""
     idx = WORKLOADS.index(name)
     g = torch.Generator(device=device).manual_seed(SEED_BASE + idx)
     if name == "dense_257":
@@ -190,7 +191,7 @@ def make(name: str, dtype=torch.bfloat16, device="cpu") -> Problem:
         return Problem(name, "dense", q, k, v, softmax_scale=1 / math.sqrt(D),
                        seqused_k=su, max_seqlen_q=Sq, max_seqlen_k=Sk)
     if name == "decode_splitkv":
-        B, Sq, Sk, Hq, Hkv, D = 8, 1, 131072, 32, 8, 128
+        B, Sq, Sk, Hq, Hkv, D = 8, 1, int(decode_sk), 32, 8, 128
         q = _randn((B, Sq, Hq, D), g, dtype)
         k = _randn((B, Sk, Hkv, D), g, dtype)
         v = _randn((B, Sk, Hkv, D), g, dtype)
