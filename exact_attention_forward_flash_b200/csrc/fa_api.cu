@@ -106,6 +106,8 @@ fa_status launch_fwd(FwdParams &p, int dev, cudaStream_t st) {
       return fail(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     configured[dev] = true;
   }
+  // causal problems with few enough sequences use the compact schedule
+  p.compact = (p.m_major && p.B >= 1 && p.B <= C::kMaxSchedB) ? 1 : 0;
   const int grid = std::min(p.num_units, num_sms(dev));
   fa_fwd_kernel<C><<<grid, C::kThreads, C::kSmemBytes, st>>>(p);
   cudaError_t e = cudaGetLastError();

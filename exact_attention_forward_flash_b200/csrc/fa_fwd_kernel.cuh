@@ -10,9 +10,12 @@
 // P.V accumulation) is the loop that "ATFlash-Kernel-FA4" (What the window
 // does) describes.
 //
-// Structure of one CTA (persistent; it walks work units u = blockIdx.x,
-// blockIdx.x + gridDim.x, ...):
+// Structure of one CTA (persistent; grid = number of SMs):
 //
+//   warp 2      tile scheduler: decodes this CTA's work units (a static snake
+//               over an ordered unit list, see decode_unit / unit_of) and
+//               publishes them, one record each, through a small ring in
+//               shared memory that the other roles read in the same order.
 //   warp 0      TMA producer: Q tiles once per unit, then K and V tiles of
 //               BN keys through separate KST-/VST-stage shared-memory rings.
 //   warp 1      MMA issuer (one thread): S = Q K^T (SS form, both operands
@@ -20,7 +23,7 @@
 //               and O += P V (TS form: P read from tensor memory where it
 //               overwrites S, V MN-major in shared memory).  Also owns the
 //               tensor-memory allocation.
-//   warps 2,3   idle.
+//   warp 3      idle.
 //   warps 4..   one 128-thread softmax warpgroup per Q tile; thread r owns
 //               tile row r (= TMEM lane r).  Per KV tile it loads its score
 //               row from tensor memory, adds the relative bias, applies the
@@ -46,6 +49,8 @@ namespace fab {
 __device__ unsigned g_fa_error;  // watchdog word, read by fa_check_device_error
 
 constexpr int kBM = 128;  // rows per Q tile = TMEM lanes
+constexpr int kUnitRing = 4;      // published units in flight
+constexpr int kUnitBytes = 64;    // one unit record in shared memory
 
 struct FwdParams {
   CUtensorMap tm_q, tm_k, tm_v;  // 3-D maps over [tokens, heads, D]
@@ -64,6 +69,7 @@ struct FwdParams {
   int split_keys;    // keys per split (multiple of BN); >= any k_len when 1 split
   int causal;
   int m_major;       // unit order: 1 = largest tile index first over all heads
+  int compact;       // 1: causal units enumerated without empty ones (see Sched)
   int lse_dense;     // 1: lse [B, Hq, Sq]; 0: lse [Hq, total_q]
   int num_units;
   float scale_log2;  // softmax_scale * log2(e)
@@ -82,15 +88,80 @@ struct Unit {
   unsigned active;   // bit t: tile t holds at least one valid row
 };
 
+// Compact heaviest-first schedule of causal units, built per CTA in shared
+// memory.  Sequences are ranked by their number of tile levels nt (a level is
+// one 256-row tile index m, over all head groups and splits); with nt sorted
+// in decreasing order, levels m in [nt[j+1], nt[j]) exist for exactly the
+// sequences of rank 0..j.  Segment j lists those levels from the top down, so
+// the whole list runs from the heaviest (largest m) unit to the lightest and
+// holds no unit without rows.
+struct Sched {
+  int *n_units;    // [1]
+  int *sorted_b;   // [B]      batch index by rank
+  int *nt;         // [B + 1]  levels of the sequence of each rank, nt[B] = 0
+  int *seg_start;  // [B + 1]  first unit of each segment
+};
+
+__device__ __forceinline__ int seq_tiles(const FwdParams &p, int b, int rows_per_unit) {
+  const int ql = p.cu_q != nullptr ? __ldg(p.cu_q + b + 1) - __ldg(p.cu_q + b) : p.Sq;
+  return ql <= 0 ? 0 : (int)(((long long)ql * p.P + rows_per_unit - 1) / rows_per_unit);
+}
+
+// Built by one warp before the CTA's first barrier.
+template <int NQ>
+__device__ __forceinline__ void build_sched(const FwdParams &p, const Sched &sch, int lane) {
+  const int B = p.B;
+  for (int b = lane; b < B; b += 32) {
+    const int nb = seq_tiles(p, b, NQ * kBM);
+    int rank = 0;
+    for (int o = 0; o < B; ++o) {
+      const int no = seq_tiles(p, o, NQ * kBM);
+      rank += (no > nb) || (no == nb && o < b);
+    }
+    sch.sorted_b[rank] = b;
+    sch.nt[rank] = nb;
+  }
+  __syncwarp();
+  if (lane == 0) {
+    sch.nt[B] = 0;
+    const int W = p.n_groups * p.num_splits;
+    int start = 0;
+    for (int j = 0; j < B; ++j) {
+      sch.seg_start[j] = start;
+      start += (sch.nt[j] - sch.nt[j + 1]) * (j + 1) * W;
+    }
+    sch.seg_start[B] = start;
+    *sch.n_units = start;
+  }
+}
+
 // Unit u -> (batch, head group, tile index, split).  Causal problems are
 // enumerated tile-index-major from the last (heaviest) tile down, so that the
 // units come roughly sorted by decreasing work across all sequences and
 // heads; other problems keep all tiles of one (batch, head group) together so
 // that concurrently running CTAs share that head's K/V in L2.
 template <int NQ, int BN>
-__device__ __forceinline__ bool decode_unit(const FwdParams &p, int u, Unit &U) {
+__device__ __forceinline__ bool decode_unit(const FwdParams &p, const Sched &sch, int u, Unit &U) {
   int mblk, grp;
-  if (p.m_major) {
+  if (p.compact) {
+    int lo = 0, hi = p.B - 1;  // last segment starting at or before u
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (sch.seg_start[mid] <= u) lo = mid; else hi = mid - 1;
+    }
+    const int j = lo;
+    const int W = p.n_groups * p.num_splits;
+    const int per_level = (j + 1) * W;
+    const int local = u - sch.seg_start[j];
+    const int lvl = local / per_level;
+    mblk = sch.nt[j] - 1 - lvl;
+    int rem = local - lvl * per_level;
+    const int bi = rem / W;
+    U.b = sch.sorted_b[bi];
+    rem -= bi * W;
+    U.split = rem % p.num_splits;
+    grp = rem / p.num_splits;
+  } else if (p.m_major) {
     const int per_m = p.B * p.n_groups * p.num_splits;
     const int m_rev = u / per_m;
     int rest = u - m_rev * per_m;
@@ -194,9 +265,18 @@ struct FwdCfg {
   static constexpr int bQFull = 0, bQEmpty = NQ, bKFull = 2 * NQ, bKEmpty = bKFull + KST,
                        bVFull = bKEmpty + KST, bVEmpty = bVFull + VST, bSFull = bVEmpty + VST,
                        bPFull = bSFull + NQ * NS, bOFull = bPFull + NQ * NS,
-                       bOEmpty = bOFull + NQ * NS, bDrain = bOEmpty + NQ, kNumBars = bDrain + 1;
+                       bOEmpty = bOFull + NQ * NS, bDrain = bOEmpty + NQ,
+                       bUFull = bDrain + 1, bUEmpty = bUFull + kUnitRing,
+                       kNumBars = bUEmpty + kUnitRing;
+  // consumers of each published unit: producer, MMA issuer, every softmax warp
+  static constexpr uint32_t kUnitConsumers = 2 + 4 * NQ;
   static constexpr int kSlotOff = kBarOff + kNumBars * 8;
-  static constexpr int kSmemBytes = kSlotOff + 16 + 1024;  // + alignment slack
+  // compact causal schedule: 3 int arrays of up to kMaxSchedB + 1 entries
+  static constexpr int kSchedOff = kSlotOff + 16;
+  static constexpr int kSchedRoom = 232448 - 1024 - kSchedOff - 16 - 16 - kUnitRing * kUnitBytes;
+  static constexpr int kMaxSchedB = (kSchedRoom / 12 - 1) > 256 ? 256 : (kSchedRoom / 12 - 1);
+  static constexpr int kRingOff = (kSchedOff + 16 + 12 * (kMaxSchedB + 1) + 15) / 16 * 16;
+  static constexpr int kSmemBytes = kRingOff + kUnitRing * kUnitBytes + 1024;  // + alignment slack
   static constexpr int kThreads = 128 * (1 + NQ);
   // registers: with two softmax warpgroups the launch budget (65536 / 384
   // threads = 168 each) is re-split so that the softmax warps hold a whole
@@ -214,6 +294,80 @@ struct FwdCfg {
 };
 
 // ---------------------------------------------------------------------------
+// unit ring: the scheduler warp decodes each unit once and publishes it;
+// producer, MMA issuer and softmax warps read the same sequence
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void unit_store(uint32_t addr, const Unit &U) {
+  sts_v4(addr, make_uint4(U.b, U.hq0, U.hk, U.split));
+  sts_v4(addr + 16, make_uint4(U.q_start, U.q_len, U.k_start, U.k_len));
+  sts_v4(addr + 32, make_uint4(U.delta, U.row0, U.kv_lo, U.kv_hi));
+  sts_v4(addr + 48, make_uint4(U.nb, U.active, 0u, 0u));
+}
+
+__device__ __forceinline__ void unit_load(uint32_t addr, Unit &U) {
+  uint4 a = lds_v4(addr), b = lds_v4(addr + 16), c = lds_v4(addr + 32), d = lds_v4(addr + 48);
+  U.b = a.x; U.hq0 = a.y; U.hk = a.z; U.split = a.w;
+  U.q_start = b.x; U.q_len = b.y; U.k_start = b.z; U.k_len = b.w;
+  U.delta = c.x; U.row0 = c.y; U.kv_lo = c.z; U.kv_hi = c.w;
+  U.nb = (int)d.x; U.active = d.y;
+}
+
+// Next unit for one consumer.  `warp_wide`: all 32 lanes read and one
+// arrival per warp is made; otherwise the calling thread alone.  Returns
+// false at the end of the schedule (a record with nb < 0) or on a timeout
+// (then *ok is false).
+template <class C>
+__device__ __forceinline__ bool next_unit(const FwdParams &p, uint32_t sb, uint32_t &cnt, Unit &U,
+                                          bool &ok, bool warp_wide) {
+  const uint32_t slot = cnt % kUnitRing;
+  const uint32_t full = sb + C::kBarOff + 8u * (C::bUFull + slot);
+  bool w = mbar_wait(full, (cnt / kUnitRing) & 1u, &g_fa_error, p.timeout_ns);
+  if (warp_wide) w = __all_sync(0xffffffffu, w);
+  if (!w) {
+    ok = false;
+    return false;
+  }
+  unit_load(sb + C::kRingOff + slot * kUnitBytes, U);
+  if (warp_wide) __syncwarp();
+  if (!warp_wide || (threadIdx.x & 31u) == 0)
+    mbar_arrive(sb + C::kBarOff + 8u * (C::bUEmpty + slot));
+  ++cnt;
+  return U.nb >= 0;
+}
+
+template <class C>
+__device__ __forceinline__ void role_scheduler(const FwdParams &p, const Sched &sch, uint32_t sb) {
+  uint32_t cnt = 0;
+  auto publish = [&](const Unit &U) -> bool {
+    const uint32_t slot = cnt % kUnitRing;
+    if (!mbar_wait_sleepy(sb + C::kBarOff + 8u * (C::bUEmpty + slot),
+                          ((cnt / kUnitRing) & 1u) ^ 1u, &g_fa_error, p.timeout_ns))
+      return false;
+    unit_store(sb + C::kRingOff + slot * kUnitBytes, U);
+    mbar_arrive(sb + C::kBarOff + 8u * (C::bUFull + slot));
+    ++cnt;
+    return true;
+  };
+  const int n_units = p.compact ? *sch.n_units : p.num_units;
+  bool ok = true;
+  for (int k = 0; k * (int)gridDim.x < n_units && ok; ++k) {
+    const int u = unit_of(k);
+    Unit U;
+    if (u >= n_units || !decode_unit<C::NQ, C::BN>(p, sch, u, U)) continue;
+    ok = publish(U);
+  }
+  if (ok) {
+    Unit end;
+    end.b = end.hq0 = end.hk = end.split = 0;
+    end.q_start = end.q_len = end.k_start = end.k_len = end.delta = end.row0 = 0;
+    end.kv_lo = end.kv_hi = 0;
+    end.nb = -1;
+    end.active = 0u;
+    publish(end);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // producer
 // ---------------------------------------------------------------------------
 template <class C>
@@ -224,10 +378,10 @@ __device__ __forceinline__ void role_producer(const FwdParams &p, uint32_t sb) {
   for (int t = 0; t < C::NQ; ++t) q_cnt[t] = 0;
   uint32_t k_cnt = 0, v_cnt = 0;
   bool ok = true;
-  for (int k = 0; k * (int)gridDim.x < p.num_units && ok; ++k) {
-    const int u = unit_of(k);
-    Unit U;
-    if (u >= p.num_units || !decode_unit<C::NQ, C::BN>(p, u, U) || U.nb == 0) continue;
+  uint32_t ucnt = 0;
+  Unit U;
+  while (ok && next_unit<C>(p, sb, ucnt, U, ok, false)) {
+    if (U.nb == 0) continue;
 #pragma unroll
     for (int t = 0; t < C::NQ; ++t) {
       if (!(U.active >> t & 1u)) continue;
@@ -324,10 +478,10 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
     tc_commit(bar(C::bOFull + t * C::NS + g % C::NS));
   };
 
-  for (int k = 0; k * (int)gridDim.x < p.num_units && ok; ++k) {
-    const int u = unit_of(k);
-    Unit U;
-    if (u >= p.num_units || !decode_unit<C::NQ, C::BN>(p, u, U) || U.nb == 0) continue;
+  uint32_t ucnt = 0;
+  Unit U;
+  while (ok && next_unit<C>(p, sb, ucnt, U, ok, false)) {
+    if (U.nb == 0) continue;
     const int nb = U.nb;
     const int last_t = (U.active >> 1 & 1u) && C::NQ > 1 ? 1 : 0;
     uint32_t sbase[C::NQ];
@@ -521,10 +675,10 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
   uint32_t s_cnt = 0;
   bool ok = true;
 
-  for (int k = 0; k * (int)gridDim.x < p.num_units && ok; ++k) {
-    const int u = unit_of(k);
-    Unit U;
-    if (u >= p.num_units || !decode_unit<C::NQ, BN>(p, u, U) || !(U.active >> t & 1u)) continue;
+  uint32_t ucnt = 0;
+  Unit U;
+  while (ok && next_unit<C>(p, sb, ucnt, U, ok, true)) {
+    if (!(U.active >> t & 1u)) continue;
     const int row = U.row0 + t * kBM + tid;
     const int i = row >> p.lgP;
     const int h = U.hq0 + (row & (p.P - 1));
@@ -867,6 +1021,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) fa_fwd_kernel(const __grid_con
       uint32_t cnt = 1;
       if (b >= C::bPFull && b < C::bPFull + C::NQ * C::NS) cnt = 128;
       if (b >= C::bOEmpty && b < C::bOEmpty + C::NQ) cnt = 128;
+      if (b >= C::bUEmpty && b < C::bUEmpty + kUnitRing) cnt = C::kUnitConsumers;
       mbar_init(sb + C::kBarOff + 8u * b, cnt);
     }
     fence_mbar_init();
@@ -878,6 +1033,15 @@ __global__ void __launch_bounds__(C::kThreads, 1) fa_fwd_kernel(const __grid_con
     tmem_alloc(sb + C::kSlotOff, C::kTmemCols);
     tmem_relinquish();
   }
+  Sched sch;
+  {
+    int *base = reinterpret_cast<int *>(smem + C::kSchedOff);
+    sch.n_units = base;
+    sch.sorted_b = base + 4;
+    sch.nt = sch.sorted_b + (C::kMaxSchedB + 1);
+    sch.seg_start = sch.nt + (C::kMaxSchedB + 1);
+  }
+  if (warp == 2 && p.compact) build_sched<C::NQ>(p, sch, lane);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -889,6 +1053,8 @@ __global__ void __launch_bounds__(C::kThreads, 1) fa_fwd_kernel(const __grid_con
       if (lane == 0) role_producer<C>(p, sb);
     } else if (warp == 1) {
       if (lane == 0) role_mma<C>(p, sb, tmem);
+    } else if (warp == 2) {
+      if (lane == 0) role_scheduler<C>(p, sch, sb);
     }
   } else {
     if constexpr (C::kSplitRegs) regs_raise<C::kRegsSoftmax>();

@@ -97,6 +97,26 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
+// Bounded wait for threads off the critical path: backs off with a short
+// sleep between polls so that it takes few issue slots from the warps that
+// share its scheduler.
+__device__ __forceinline__ bool mbar_wait_sleepy(uint32_t bar, uint32_t parity, unsigned *err,
+                                                 uint64_t timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(256);
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 15u) == 0) {
+      if (*reinterpret_cast<volatile unsigned *>(err) != 0u) return false;
+      if (global_timer_ns() - t0 > timeout_ns) {
+        atomicOr(err, kErrTimeout);
+        return false;
+      }
+    }
+  }
+}
+
 // Drain wait used after a timeout: ignores the error word (work already in
 // flight must land before shared or tensor memory is released) but is still
 // bounded by `timeout_ns`.
