@@ -252,13 +252,23 @@ def time_steps(step, steps: int, warmup: int, dist_on: bool, device_index: int):
 
 
 def max_over_ranks(x: float, dist_on: bool) -> float:
+    """The maximum of a per-rank time over all ranks (NCCL on the GPU, or a
+    CPU tensor when the process group runs on gloo)."""
     if not dist_on:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_value(per_rank_units: float, world: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank processes its own copy of the
+    workload, so the units of all ranks are divided by the slowest rank's
+    time (in ms), giving units per second."""
+    return world * per_rank_units / (max_ms * 1e-3)
 
 
 def roofline(p, per_launch_ms: float, peaks, traffic):
@@ -356,8 +366,9 @@ def main():
     total_ms, per_ms, clocks = time_steps(run, a.steps, a.warmup, dist_on, local)
     total_ms = max_over_ranks(total_ms, dist_on)
     ms_step = total_ms / a.steps
-    value = world * workload_value(p, ms_step)[0]
     unit = workload_value(p, ms_step)[1]
+    per_rank_units = p.hbm_bytes() / 1e9 if p.splitkv else p.flops() / 1e12
+    value = weak_value(per_rank_units, world, ms_step)  # TFLOP/s or GB/s
     traffic = profiled_traffic(a.workload)
     roof = roofline(p, per_ms, peaks, traffic)
 

@@ -1,0 +1,68 @@
+"""The multi-GPU protocol of bench.py, exercised on CPU with gloo ranks.
+
+Each rank of a weak-scaling run processes its own copy of the workload; the
+job's time is the slowest rank's device time (max over ranks) and the value
+divides the units of all ranks by it.  These tests run two gloo ranks on the
+host (no GPU) and check that reduction, and that the reference arm leaves
+the work to rank 0.
+"""
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, times, out_q):
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        mx = bench.max_over_ranks(times[rank], True)
+        val = bench.weak_value(1e12, world, mx)
+        dist.barrier()
+        out_q.put((rank, mx, val))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_with_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    times = [3.5, 7.25]
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, times, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, mx, val in res:
+        assert mx == 7.25
+        # 2 ranks x 1e12 units over 7.25 ms
+        assert val == pytest.approx(2 * 1e12 / 7.25e-3)
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    env = dict(os.environ, WORLD_SIZE="2", RANK="1", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "0"], env=env, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""
