@@ -50,10 +50,52 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Encoded maps are cached per host thread (a call encodes three, and the
+// driver call dominates the host cost of small problems); the key is every
+// input of the encoding.
+struct MapKey {
+  const void *base;
+  long long tokens;
+  int D, H, box_h, box_t, half;
+  bool operator==(const MapKey &o) const {
+    return base == o.base && tokens == o.tokens && D == o.D && H == o.H && box_h == o.box_h &&
+           box_t == o.box_t && half == o.half;
+  }
+};
+constexpr int kMapCache = 16;
+struct MapCache {
+  MapKey key[kMapCache];
+  CUtensorMap map[kMapCache];
+  bool used[kMapCache] = {};
+  int next = 0;
+};
+thread_local MapCache g_maps;
+
+fa_status encode_map(CUtensorMap *tm, const void *base, int D, int H, long long tokens, int box_h,
+                     int box_t, bool half);
+
 // 3-D map over a [tokens, heads, D] tensor of 16-bit elements with a box of
 // {64 columns, box_h heads, box_t tokens}, 128-byte swizzle, zero fill.
 fa_status make_map(CUtensorMap *tm, const void *base, int D, int H, long long tokens, int box_h,
                    int box_t, bool half) {
+  const MapKey k{base, tokens, D, H, box_h, box_t, half ? 1 : 0};
+  for (int i = 0; i < kMapCache; ++i)
+    if (g_maps.used[i] && g_maps.key[i] == k) {
+      *tm = g_maps.map[i];
+      return FA_OK;
+    }
+  fa_status s = encode_map(tm, base, D, H, tokens, box_h, box_t, half);
+  if (s != FA_OK) return s;
+  const int i = g_maps.next;
+  g_maps.next = (i + 1) % kMapCache;
+  g_maps.key[i] = k;
+  g_maps.map[i] = *tm;
+  g_maps.used[i] = true;
+  return FA_OK;
+}
+
+fa_status encode_map(CUtensorMap *tm, const void *base, int D, int H, long long tokens, int box_h,
+                     int box_t, bool half) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)tokens};
@@ -88,8 +130,8 @@ int num_sms(int dev) {
 // kernel variants
 using Fwd128B = FwdCfg<128, 128, 2, 1, 2, 2, false, false>;
 using Fwd128H = FwdCfg<128, 128, 2, 1, 2, 2, true, false>;
-using Fwd256B = FwdCfg<256, 64, 1, 2, 2, 2, false, false>;
-using Fwd256H = FwdCfg<256, 64, 1, 2, 2, 2, true, false>;
+using Fwd256B = FwdCfg<256, 64, 1, 2, 3, 2, false, false>;
+using Fwd256H = FwdCfg<256, 64, 1, 2, 3, 2, true, false>;
 using Spl128B = FwdCfg<128, 128, 1, 2, 3, 3, false, true>;
 using Spl128H = FwdCfg<128, 128, 1, 2, 3, 3, true, true>;
 using Spl256B = FwdCfg<256, 64, 1, 2, 2, 2, false, true>;

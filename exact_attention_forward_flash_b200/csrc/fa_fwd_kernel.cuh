@@ -49,6 +49,19 @@ namespace fab {
 __device__ unsigned g_fa_error;  // watchdog word, read by fa_check_device_error
 
 constexpr int kBM = 128;  // rows per Q tile = TMEM lanes
+
+// Every kEmuPeriod-th column's exponential runs on the FMA pipe (ex2_poly)
+// rather than the MUFU unit, which is otherwise as loaded as the tensor core.
+#ifndef FA_EMU_PERIOD
+#define FA_EMU_PERIOD 0
+#endif
+constexpr int kEmuPeriod = FA_EMU_PERIOD;
+__device__ __forceinline__ constexpr bool emulated_exp(int c) {
+  return kEmuPeriod > 0 && (c % (kEmuPeriod > 0 ? kEmuPeriod : 1)) == kEmuPeriod - 1;
+}
+__device__ __forceinline__ float exp2_col(int c, float x) {
+  return emulated_exp(c) ? ex2_poly(x) : ex2_approx(x);
+}
 constexpr int kUnitRing = 4;      // published units in flight
 constexpr int kUnitBytes = 64;    // one unit record in shared memory
 
@@ -465,6 +478,7 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
     tc_commit(bar(C::bSFull + t * C::NS + g % C::NS));
   };
   // O_t += P_t(g) V (P in the S buffer of g, as 16-bit pairs)
+  // O_t += P_t(g) V (P in the S buffer of g, as 16-bit pairs)
   auto issue_pv = [&](int t, uint32_t g, uint32_t vstage, bool first) {
     const uint32_t va = sb + C::kVOff + vstage * C::kKVTile;
     const uint32_t p_tmem = tmem + C::s_col(t, g % C::NS);
@@ -866,8 +880,8 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
           uint32_t pk[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * e]), sl2, -mc));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * e + 1]), sl2, -mc));
+            const float p0 = exp2_col(2 * e, fmaf(__uint_as_float(r[2 * e]), sl2, -mc));
+            const float p1 = exp2_col(2 * e + 1, fmaf(__uint_as_float(r[2 * e + 1]), sl2, -mc));
             lsum += p0 + p1;
             pk[e] = pack2<C::HALF>(p0, p1);
           }
@@ -879,6 +893,8 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
           if (!ok) break;
           tmem_wait_st();
         }
+        tc_fence_before();
+        mbar_arrive(bar(C::bPFull + t * NS + buf));
       } else {
         ok = wait_scores();
         if (!ok) break;
@@ -909,9 +925,14 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
             for (int c = 0; c < BN; ++c)
               if (c >= lim_c) s[c] = -INFINITY;
           }
-          float mx = s[0];
+          // row max over 4 independent chains (a single chain of BN
+          // dependent max operations would be pure latency)
+          float m4[4];
 #pragma unroll
-          for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+          for (int e = 0; e < 4; ++e) m4[e] = s[e];
+#pragma unroll
+          for (int c = 4; c < BN; ++c) m4[c & 3] = fmaxf(m4[c & 3], s[c]);
+          const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
           const float m_new = fmaxf(m_ref, mx);
           if (n == 0) {
             m_ref = m_new;
@@ -929,13 +950,12 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
             }
           }
           const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * sl2;
-          float lsum = 0.f;
+          float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int c = 0; c < BN; ++c) {
-            s[c] = ex2_approx(fmaf(s[c], sl2, -mc));
-            lsum += s[c];
+            s[c] = exp2_col(c, fmaf(s[c], sl2, -mc));
+            l4[c & 3] += s[c];
           }
-          l += lsum;
 #pragma unroll
           for (int c = 0; c < BN / 64; ++c) {
             uint32_t r[32];
@@ -945,10 +965,14 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
             tmem_st32(s_addr + 32 * c, r);
           }
           tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(C::bPFull + t * NS + buf));
+          l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+        } else {
+          tc_fence_before();
+          mbar_arrive(bar(C::bPFull + t * NS + buf));
         }
       }
-      tc_fence_before();
-      mbar_arrive(bar(C::bPFull + t * NS + buf));
     }
     if (!ok) break;
 

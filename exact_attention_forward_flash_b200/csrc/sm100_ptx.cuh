@@ -293,6 +293,26 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 2^x for x <= 8 on the FMA and integer pipes instead of the MUFU unit:
+// x = j + f with j = round(x) (the 1.5 * 2^23 addition leaves round(x) in the
+// low mantissa bits), 2^f on [-1/2, 1/2] from a degree-3 polynomial fitted
+// here by a Remez exchange for minimal relative error (below 7.5e-5), and 2^j
+// applied by adding j to the exponent field.  Inputs below -126, -inf for a
+// masked key among them, give exactly 0, as the MUFU instruction does: a row
+// whose keys are all masked must keep a zero normaliser.
+__device__ __forceinline__ float ex2_poly(float x) {
+  const float xc = fmaxf(x, -126.f);
+  const float t = xc + 12582912.f;
+  const float j = t - 12582912.f;
+  const float f = xc - j;
+  const float p = fmaf(fmaf(fmaf(0.05517166905807796f, f, 0.24261112219322045f), f,
+                            0.6932609854606147f),
+                       f, 0.9999280735393961f);
+  const int e = __float_as_int(t) - 0x4B400000;
+  const float r = __int_as_float(__float_as_int(p) + (e << 23));
+  return x < -126.f ? 0.f : r;
+}
+
 __device__ __forceinline__ float lg2_approx(float x) {
   float y;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

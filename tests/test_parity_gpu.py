@@ -271,7 +271,7 @@ def test_bias_none_equals_bias_zero():
     compare(o1, l1, ro, rl, what="no bias")
     compare(o2, l2, ro, rl, what="zero bias")
     assert (o1.float() - o2.float()).abs().max().item() <= 8e-3
-    assert (l1 - l2).abs().max().item() <= 1e-5
+    assert (l1 - l2).abs().max().item() <= 1e-4
 
 
 def test_deterministic_run_to_run():
