@@ -1121,18 +1121,37 @@ __global__ void __launch_bounds__(256) fa_combine_kernel(const float *__restrict
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.f;
   if (m != -INFINITY) {
-    for (int s = 0; s < ns; ++s) {
-      const float ls = lse_part[(long long)s * rows + r];
-      if (ls == -INFINITY) continue;
-      const float w = ex2_approx((ls - Lse) * L2E);
-      const float *src = o_part + ((long long)s * rows + r) * D + lane * E;
+    // splits in groups of 8 whose loads are all issued before any is used
+    // (a weight of 0 stands for a split with no keys)
+    constexpr int U = 8;
+    for (int s0 = 0; s0 < ns; s0 += U) {
+      float w[U];
+      float4 x[U][E / 4];
 #pragma unroll
-      for (int e = 0; e < E; e += 4) {
-        const float4 x = *reinterpret_cast<const float4 *>(src + e);
-        acc[e] += w * x.x;
-        acc[e + 1] += w * x.y;
-        acc[e + 2] += w * x.z;
-        acc[e + 3] += w * x.w;
+      for (int u = 0; u < U; ++u) {
+        const int s = s0 + u;
+        w[u] = 0.f;
+        if (s < ns) {
+          const float ls = __ldg(lse_part + (long long)s * rows + r);
+          w[u] = ls == -INFINITY ? 0.f : ex2_approx((ls - Lse) * L2E);
+          const float4 *src =
+              reinterpret_cast<const float4 *>(o_part + ((long long)s * rows + r) * D + lane * E);
+#pragma unroll
+          for (int e = 0; e < E / 4; ++e) x[u][e] = __ldg(src + e);
+        } else {
+#pragma unroll
+          for (int e = 0; e < E / 4; ++e) x[u][e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+#pragma unroll
+        for (int e = 0; e < E / 4; ++e) {
+          acc[4 * e] += w[u] * x[u][e].x;
+          acc[4 * e + 1] += w[u] * x[u][e].y;
+          acc[4 * e + 2] += w[u] * x[u][e].z;
+          acc[4 * e + 3] += w[u] * x[u][e].w;
+        }
       }
     }
   }
