@@ -50,17 +50,57 @@ __device__ unsigned g_fa_error;  // watchdog word, read by fa_check_device_error
 
 constexpr int kBM = 128;  // rows per Q tile = TMEM lanes
 
-// Every kEmuPeriod-th column's exponential runs on the FMA pipe (ex2_poly)
-// rather than the MUFU unit, which is otherwise as loaded as the tensor core.
-#ifndef FA_EMU_PERIOD
-#define FA_EMU_PERIOD 0
+// Of every 8 pairs of columns, this many take their exponential on the FMA
+// pipe (ex2_poly2) rather than the MUFU unit, which at D = 128 is otherwise
+// as loaded as the tensor core (one exponential per 4*D tensor-core flops).
+#ifndef FA_POLY_PAIRS
+#define FA_POLY_PAIRS 2
 #endif
-constexpr int kEmuPeriod = FA_EMU_PERIOD;
-__device__ __forceinline__ constexpr bool emulated_exp(int c) {
-  return kEmuPeriod > 0 && (c % (kEmuPeriod > 0 ? kEmuPeriod : 1)) == kEmuPeriod - 1;
+constexpr int kPolyPairs = FA_POLY_PAIRS;
+
+// P = 2^(s * sl2 - mc) for the N columns [OFF, OFF + N) of a row, rounded to
+// 16-bit pairs into pk; returns the sum of the unrounded values.  kPoly
+// sends kPolyPairs of every 8 pairs through ex2_poly2, which needs finite
+// scores (no masked column).
+template <bool kHalf, bool kPoly, int OFF, int N, int M>
+__device__ __forceinline__ float exp_pack(const float (&s)[M], float sl2, float mc,
+                                          uint32_t (&pk)[N / 2]) {
+  const uint64_t sc = f2(sl2, sl2), nm = f2(-mc, -mc);
+  uint64_t acc0 = f2(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+  for (int q = 0; q < N / 2; ++q) {
+    float x0, x1, y0, y1;
+    f2_split(ffma2(f2(s[OFF + 2 * q], s[OFF + 2 * q + 1]), sc, nm), x0, x1);
+    if (kPoly && (q % 8) < kPolyPairs) {
+      ex2_poly2(x0, x1, y0, y1);
+    } else {
+      y0 = ex2_approx(x0);
+      y1 = ex2_approx(x1);
+    }
+    if (q & 1)
+      acc1 = fadd2(acc1, f2(y0, y1));
+    else
+      acc0 = fadd2(acc0, f2(y0, y1));
+    pk[q] = pack2<kHalf>(y0, y1);
+  }
+  float a, b, c, d;
+  f2_split(acc0, a, b);
+  f2_split(acc1, c, d);
+  return (a + b) + (c + d);
 }
-__device__ __forceinline__ float exp2_col(int c, float x) {
-  return emulated_exp(c) ? ex2_poly(x) : ex2_approx(x);
+
+// Row max of the N columns [OFF, OFF + N) over four independent chains of
+// three-input maxima.
+template <int OFF, int N, int M>
+__device__ __forceinline__ float row_max(const float (&s)[M]) {
+  float m4[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) m4[k] = fmaxf(s[OFF + 2 * k], s[OFF + 2 * k + 1]);
+#pragma unroll
+  for (int c = 8; c < N; c += 8)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m4[k] = fmax3(m4[k], s[OFF + c + 2 * k], s[OFF + c + 2 * k + 1]);
+  return fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
 }
 constexpr int kUnitRing = 4;      // published units in flight
 constexpr int kUnitBytes = 64;    // one unit record in shared memory
@@ -473,9 +513,9 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
       const uint32_t off = (kk % 4) * 32;  // 16 elements = 32 bytes inside the swizzle atom
       const uint64_t a = smem_desc_sw128(qa + (kk / 4) * C::kQChunk + off, 16, 1024);
       const uint64_t b = smem_desc_sw128(ka + (kk / 4) * C::kKVChunk + off, 16, 1024);
-      tc_mma_ss(d_tmem, a, b, idesc_s, kk > 0 ? 1u : 0u);
+      tc_mma_ss_elect(d_tmem, a, b, idesc_s, kk > 0 ? 1u : 0u);
     }
-    tc_commit(bar(C::bSFull + t * C::NS + g % C::NS));
+    tc_commit_elect(bar(C::bSFull + t * C::NS + g % C::NS));
   };
   // O_t += P_t(g) V (P in the S buffer of g, as 16-bit pairs)
   // O_t += P_t(g) V (P in the S buffer of g, as 16-bit pairs)
@@ -487,14 +527,14 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
     for (int kk = 0; kk < C::BN / 16; ++kk) {
       // 16 keys = two 8-row groups (SBO 1024 B); 64-column chunks LBO apart
       const uint64_t b = smem_desc_sw128(va + kk * 16 * 128, C::kKVChunk, 1024);
-      tc_mma_ts(d_tmem, p_tmem + kk * 8, b, idesc_pv, (first && kk == 0) ? 0u : 1u);
+      tc_mma_ts_elect(d_tmem, p_tmem + kk * 8, b, idesc_pv, (first && kk == 0) ? 0u : 1u);
     }
-    tc_commit(bar(C::bOFull + t * C::NS + g % C::NS));
+    tc_commit_elect(bar(C::bOFull + t * C::NS + g % C::NS));
   };
 
   uint32_t ucnt = 0;
   Unit U;
-  while (ok && next_unit<C>(p, sb, ucnt, U, ok, false)) {
+  while (ok && next_unit<C>(p, sb, ucnt, U, ok, true)) {
     if (U.nb == 0) continue;
     const int nb = U.nb;
     const int last_t = (U.active >> 1 & 1u) && C::NQ > 1 ? 1 : 0;
@@ -503,7 +543,7 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
     for (int t = 0; t < C::NQ; ++t) {
       sbase[t] = s_cnt[t];
       if (!(U.active >> t & 1u)) continue;
-      ok = ok && mbar_wait(bar(C::bQFull + t), q_cnt[t] & 1u, &g_fa_error, p.timeout_ns);
+      ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(C::bQFull + t), q_cnt[t] & 1u, &g_fa_error, p.timeout_ns));
       ++q_cnt[t];
     }
     if (!ok) break;
@@ -511,60 +551,60 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
     const uint32_t kb = k_cnt, vb = v_cnt;
 
     // prologue: S(0) for every active tile
-    ok = mbar_wait(bar(C::bKFull + kb % C::KST), (kb / C::KST) & 1u, &g_fa_error, p.timeout_ns);
+    ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + kb % C::KST), (kb / C::KST) & 1u, &g_fa_error, p.timeout_ns));
     if (!ok) break;
     tc_fence_after();
 #pragma unroll
     for (int t = 0; t < C::NQ; ++t) {
       if (!(U.active >> t & 1u)) continue;
       issue_s(t, sbase[t], kb % C::KST);
-      if (nb == 1) tc_commit(bar(C::bQEmpty + t));
+      if (nb == 1) tc_commit_elect(bar(C::bQEmpty + t));
     }
-    tc_commit(bar(C::bKEmpty + kb % C::KST));
+    tc_commit_elect(bar(C::bKEmpty + kb % C::KST));
 
     for (int n = 0; n < nb && ok; ++n) {
       const uint32_t kn = kb + n + 1;  // K tile of block n+1
       if (C::NS == 2 && n + 1 < nb) {
-        ok = mbar_wait(bar(C::bKFull + kn % C::KST), (kn / C::KST) & 1u, &g_fa_error,
-                       p.timeout_ns);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + kn % C::KST), (kn / C::KST) & 1u, &g_fa_error,
+                       p.timeout_ns));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
         for (int t = 0; t < C::NQ; ++t) {
           if (!(U.active >> t & 1u)) continue;
           issue_s(t, sbase[t] + n + 1, kn % C::KST);
-          if (n + 1 == nb - 1) tc_commit(bar(C::bQEmpty + t));
+          if (n + 1 == nb - 1) tc_commit_elect(bar(C::bQEmpty + t));
         }
-        tc_commit(bar(C::bKEmpty + kn % C::KST));
+        tc_commit_elect(bar(C::bKEmpty + kn % C::KST));
       }
       const uint32_t vn = vb + n;
-      ok = mbar_wait(bar(C::bVFull + vn % C::VST), (vn / C::VST) & 1u, &g_fa_error,
-                     p.timeout_ns);
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bVFull + vn % C::VST), (vn / C::VST) & 1u, &g_fa_error,
+                     p.timeout_ns));
       if (!ok) break;
 #pragma unroll
       for (int t = 0; t < C::NQ; ++t) {
         if (!(U.active >> t & 1u)) continue;
         const uint32_t g = sbase[t] + n;
         if (n == 0) {
-          ok = mbar_wait(bar(C::bOEmpty + t), (u_cnt[t] & 1u) ^ 1u, &g_fa_error, p.timeout_ns);
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bOEmpty + t), (u_cnt[t] & 1u) ^ 1u, &g_fa_error, p.timeout_ns));
           if (!ok) break;
         }
-        ok = mbar_wait(bar(C::bPFull + t * C::NS + g % C::NS), (g / C::NS) & 1u, &g_fa_error,
-                       p.timeout_ns);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bPFull + t * C::NS + g % C::NS), (g / C::NS) & 1u, &g_fa_error,
+                       p.timeout_ns));
         if (!ok) break;
         tc_fence_after();
         issue_pv(t, g, vn % C::VST, n == 0);
-        if (t == last_t) tc_commit(bar(C::bVEmpty + vn % C::VST));
+        if (t == last_t) tc_commit_elect(bar(C::bVEmpty + vn % C::VST));
         if (C::NS == 1 && n + 1 < nb) {
           if (t == 0) {
-            ok = mbar_wait(bar(C::bKFull + kn % C::KST), (kn / C::KST) & 1u, &g_fa_error,
-                           p.timeout_ns);
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + kn % C::KST), (kn / C::KST) & 1u, &g_fa_error,
+                           p.timeout_ns));
             if (!ok) break;
             tc_fence_after();
           }
           issue_s(t, g + 1, kn % C::KST);
-          if (n + 1 == nb - 1) tc_commit(bar(C::bQEmpty + t));
-          if (t == last_t) tc_commit(bar(C::bKEmpty + kn % C::KST));
+          if (n + 1 == nb - 1) tc_commit_elect(bar(C::bQEmpty + t));
+          if (t == last_t) tc_commit_elect(bar(C::bKEmpty + kn % C::KST));
         }
       }
     }
@@ -578,7 +618,7 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
     }
   }
   // Wait for every MMA this thread issued before tensor memory is released.
-  tc_commit(bar(C::bDrain));
+  tc_commit_elect(bar(C::bDrain));
   mbar_wait_drain(bar(C::bDrain), 0, ok ? p.timeout_ns : 200000000ull);
 }
 
@@ -746,6 +786,9 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
                                                         base - (BN - 1) < p.R);
       const uint32_t s_addr = tmem + lane_addr + C::s_col(t, buf);
       const int lim_c = lim_rel - jrel;  // columns at or past lim_c are masked
+      // no row of the warp has a masked column here: the FMA-pipe exponential
+      // may stand in for some of the MUFU ones
+      const bool poly_ok = __all_sync(0xffffffffu, lim_c >= BN);
       auto wait_scores = [&]() -> bool {
         const bool w = __all_sync(0xffffffffu,
                                   mbar_wait(bar(C::bSFull + t * NS + buf), (g / NS) & 1u,
@@ -794,7 +837,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
           const bool staged = true;
 #pragma unroll
         for (int hf = 0; hf < BN / 64; ++hf) {
-          uint32_t r[64];
+          float x[64];
           {
             uint32_t r0[32], r1[32];
             tmem_ld32(s_addr + 64 * hf, r0);
@@ -802,25 +845,24 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              r[e] = r0[e];
-              r[32 + e] = r1[e];
+              x[e] = __uint_as_float(r0[e]);
+              x[32 + e] = __uint_as_float(r1[e]);
             }
           }
           if constexpr (C::kBiasSmem) {
             if (staged) {
               const int sh = (base - 15) & 7;  // misalignment of the bias run
+              const uint64_t isc = f2(p.inv_scale, p.inv_scale);
 #pragma unroll
               for (int cc = 0; cc < 4; ++cc) {
                 if (need >> (4 * hf + cc) & 1u) {
                   uint32_t w2[8];
                   bias_chunk<C>(bias_buf, lane, sh, pf[cc], w2);
 #pragma unroll
-                  for (int e = 0; e < 8; ++e) {
-                    r[16 * cc + 2 * e] = __float_as_uint(fmaf(
-                        lo_f<C::HALF>(w2[e]), p.inv_scale, __uint_as_float(r[16 * cc + 2 * e])));
-                    r[16 * cc + 2 * e + 1] = __float_as_uint(fmaf(
-                        hi_f<C::HALF>(w2[e]), p.inv_scale, __uint_as_float(r[16 * cc + 2 * e + 1])));
-                  }
+                  for (int e = 0; e < 8; ++e)
+                    f2_split(ffma2(f2(lo_f<C::HALF>(w2[e]), hi_f<C::HALF>(w2[e])), isc,
+                                   f2(x[16 * cc + 2 * e], x[16 * cc + 2 * e + 1])),
+                             x[16 * cc + 2 * e], x[16 * cc + 2 * e + 1]);
                 }
               }
               if (hf + 1 < BN / 64) bias_load<C, 4>(p, bf, jrel, lane, need, pf);
@@ -831,21 +873,17 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
 #pragma unroll
               for (int e = 0; e < 64; ++e) {
                 const int d = base - (64 * hf + e);
-                if (d >= 0 && d < p.R)
-                  r[e] = __float_as_uint(__uint_as_float(r[e]) +
-                                         load_elem<C::HALF>(brow + d) * p.inv_scale);
+                if (d >= 0 && d < p.R) x[e] += load_elem<C::HALF>(brow + d) * p.inv_scale;
               }
             }
           }
-          float mx = -INFINITY;
+          if (lim_c < 64 * hf + 64) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e) {
-            const float x = (64 * hf + e >= lim_c) ? -INFINITY : __uint_as_float(r[e]);
-            r[e] = __float_as_uint(x);
-            mx = fmaxf(mx, x);
+            for (int e = 0; e < 64; ++e)
+              if (64 * hf + e >= lim_c) x[e] = -INFINITY;
           }
           // running-max update with conditional rescaling
-          const float m_new = fmaxf(m_ref, mx);
+          const float m_new = fmaxf(m_ref, row_max<0, 64>(x));
           if (n == 0 && hf == 0) {
             m_ref = m_new;
           } else {
@@ -876,16 +914,11 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
             }
           }
           const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * sl2;
-          float lsum = 0.f;
           uint32_t pk[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float p0 = exp2_col(2 * e, fmaf(__uint_as_float(r[2 * e]), sl2, -mc));
-            const float p1 = exp2_col(2 * e + 1, fmaf(__uint_as_float(r[2 * e + 1]), sl2, -mc));
-            lsum += p0 + p1;
-            pk[e] = pack2<C::HALF>(p0, p1);
-          }
-          l += lsum;
+          if (kPolyPairs > 0 && poly_ok)
+            l += exp_pack<C::HALF, true, 0, 64>(x, sl2, mc, pk);
+          else
+            l += exp_pack<C::HALF, false, 0, 64>(x, sl2, mc, pk);
           // P half hf -> columns [32 hf, 32 hf + 32): only score columns
           // already read are overwritten
           tmem_st32(s_addr + 32 * hf, pk);
@@ -894,7 +927,8 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
           tmem_wait_st();
         }
         tc_fence_before();
-        mbar_arrive(bar(C::bPFull + t * NS + buf));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::bPFull + t * NS + buf));
       } else {
         ok = wait_scores();
         if (!ok) break;
@@ -925,15 +959,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
             for (int c = 0; c < BN; ++c)
               if (c >= lim_c) s[c] = -INFINITY;
           }
-          // row max over 4 independent chains (a single chain of BN
-          // dependent max operations would be pure latency)
-          float m4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) m4[e] = s[e];
-#pragma unroll
-          for (int c = 4; c < BN; ++c) m4[c & 3] = fmaxf(m4[c & 3], s[c]);
-          const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-          const float m_new = fmaxf(m_ref, mx);
+          const float m_new = fmaxf(m_ref, row_max<0, BN>(s));
           if (n == 0) {
             m_ref = m_new;
           } else {
@@ -950,27 +976,30 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
             }
           }
           const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * sl2;
-          float l4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            s[c] = exp2_col(c, fmaf(s[c], sl2, -mc));
-            l4[c & 3] += s[c];
+          {
+            uint32_t pk[32];
+            if (kPolyPairs > 0 && poly_ok)
+              l += exp_pack<C::HALF, true, 0, 64>(s, sl2, mc, pk);
+            else
+              l += exp_pack<C::HALF, false, 0, 64>(s, sl2, mc, pk);
+            tmem_st32(s_addr, pk);
           }
-#pragma unroll
-          for (int c = 0; c < BN / 64; ++c) {
-            uint32_t r[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              r[e] = pack2<C::HALF>(s[64 * c + 2 * e], s[64 * c + 2 * e + 1]);
-            tmem_st32(s_addr + 32 * c, r);
+          if constexpr (BN == 128) {
+            uint32_t pk[32];
+            if (kPolyPairs > 0 && poly_ok)
+              l += exp_pack<C::HALF, true, 64, 64>(s, sl2, mc, pk);
+            else
+              l += exp_pack<C::HALF, false, 64, 64>(s, sl2, mc, pk);
+            tmem_st32(s_addr + 32, pk);
           }
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(bar(C::bPFull + t * NS + buf));
-          l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(C::bPFull + t * NS + buf));
         } else {
           tc_fence_before();
-          mbar_arrive(bar(C::bPFull + t * NS + buf));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(C::bPFull + t * NS + buf));
         }
       }
     }
@@ -1043,7 +1072,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) fa_fwd_kernel(const __grid_con
   if (warp == 0 && lane == 0) {
     for (int b = 0; b < C::kNumBars; ++b) {
       uint32_t cnt = 1;
-      if (b >= C::bPFull && b < C::bPFull + C::NQ * C::NS) cnt = 128;
+      if (b >= C::bPFull && b < C::bPFull + C::NQ * C::NS) cnt = 4;  // one per warp
       if (b >= C::bOEmpty && b < C::bOEmpty + C::NQ) cnt = 128;
       if (b >= C::bUEmpty && b < C::bUEmpty + kUnitRing) cnt = C::kUnitConsumers;
       mbar_init(sb + C::kBarOff + 8u * b, cnt);
@@ -1076,7 +1105,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) fa_fwd_kernel(const __grid_con
     if (warp == 0) {
       if (lane == 0) role_producer<C>(p, sb);
     } else if (warp == 1) {
-      if (lane == 0) role_mma<C>(p, sb, tmem);
+      role_mma<C>(p, sb, tmem);  // whole warp; MMAs issued by the elected lane
     } else if (warp == 2) {
       if (lane == 0) role_scheduler<C>(p, sch, sb);
     }

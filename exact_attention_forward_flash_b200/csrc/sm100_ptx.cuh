@@ -178,6 +178,37 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
       : "memory");
 }
 
+// Forms issued by the elected (lowest active) lane of a converged warp: the
+// whole warp runs the issuing loop and never diverges around the issue.  The
+// same lane is elected every time, so a commit tracks the MMAs it issued.
+__device__ __forceinline__ void tc_commit_elect(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tc_mma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tc_mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // D[tmem] (+)= A[smem desc] * B[smem desc]
 __device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                           uint32_t idesc, uint32_t accumulate) {
@@ -311,6 +342,54 @@ __device__ __forceinline__ float ex2_poly(float x) {
   const int e = __float_as_int(t) - 0x4B400000;
   const float r = __int_as_float(__float_as_int(p) + (e << 23));
   return x < -126.f ? 0.f : r;
+}
+
+// --- packed fp32 pairs (sm_100 f32x2 instructions: one issue slot per pair)
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// max of three floats in one instruction (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair of finite x in [-126, 8] on the FMA and integer pipes, the
+// same construction as ex2_poly with the floating-point steps packed in
+// pairs.  Callers clamp: below -126 the result is 2^-126 rather than 0, so a
+// tile with masked (-inf) scores must not take this path.
+__device__ __forceinline__ void ex2_poly2(float x0, float x1, float &y0, float &y1) {
+  const uint64_t xc = f2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t t = fadd2(xc, f2(12582912.f, 12582912.f));
+  const uint64_t j = fadd2(t, f2(-12582912.f, -12582912.f));
+  const uint64_t f = ffma2(j, f2(-1.f, -1.f), xc);
+  uint64_t q = ffma2(f, f2(0.05517166905807796f, 0.05517166905807796f),
+                     f2(0.24261112219322045f, 0.24261112219322045f));
+  q = ffma2(q, f, f2(0.6932609854606147f, 0.6932609854606147f));
+  q = ffma2(q, f, f2(0.9999280735393961f, 0.9999280735393961f));
+  float t0, t1, q0, q1;
+  f2_split(t, t0, t1);
+  f2_split(q, q0, q1);
+  // (bits of t) << 23 leaves round(x) << 23: the 1.5 * 2^23 offset's own
+  // bits all shift out of the word
+  y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
 __device__ __forceinline__ float lg2_approx(float x) {
