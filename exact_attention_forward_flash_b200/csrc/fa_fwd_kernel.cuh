@@ -393,11 +393,15 @@ __device__ __forceinline__ void role_scheduler(const FwdParams &p, const Sched &
   uint32_t cnt = 0;
   auto publish = [&](const Unit &U) -> bool {
     const uint32_t slot = cnt % kUnitRing;
-    if (!mbar_wait_sleepy(sb + C::kBarOff + 8u * (C::bUEmpty + slot),
-                          ((cnt / kUnitRing) & 1u) ^ 1u, &g_fa_error, p.timeout_ns))
+    if (!__all_sync(0xffffffffu, mbar_wait_sleepy(sb + C::kBarOff + 8u * (C::bUEmpty + slot),
+                                                  ((cnt / kUnitRing) & 1u) ^ 1u, &g_fa_error,
+                                                  p.timeout_ns)))
       return false;
-    unit_store(sb + C::kRingOff + slot * kUnitBytes, U);
-    mbar_arrive(sb + C::kBarOff + 8u * (C::bUFull + slot));
+    if ((threadIdx.x & 31u) == 0) {  // the warp stays converged; lane 0 publishes
+      unit_store(sb + C::kRingOff + slot * kUnitBytes, U);
+      mbar_arrive(sb + C::kBarOff + 8u * (C::bUFull + slot));
+    }
+    __syncwarp();
     ++cnt;
     return true;
   };
@@ -431,53 +435,63 @@ __device__ __forceinline__ void role_producer(const FwdParams &p, uint32_t sb) {
   for (int t = 0; t < C::NQ; ++t) q_cnt[t] = 0;
   uint32_t k_cnt = 0, v_cnt = 0;
   bool ok = true;
+  const bool leader = (threadIdx.x & 31u) == 0;  // issues the copies; the warp stays converged
   uint32_t ucnt = 0;
   Unit U;
-  while (ok && next_unit<C>(p, sb, ucnt, U, ok, false)) {
+  while (ok && next_unit<C>(p, sb, ucnt, U, ok, true)) {
     if (U.nb == 0) continue;
 #pragma unroll
     for (int t = 0; t < C::NQ; ++t) {
       if (!(U.active >> t & 1u)) continue;
-      ok = mbar_wait(bar(C::bQEmpty + t), (q_cnt[t] & 1u) ^ 1u, &g_fa_error, p.timeout_ns);
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bQEmpty + t), (q_cnt[t] & 1u) ^ 1u, &g_fa_error, p.timeout_ns));
       if (!ok) break;
-      mbar_arrive_expect_tx(bar(C::bQFull + t), C::kQTile);
       const int tok = U.q_start + (U.row0 + t * kBM) / p.P;
+      if (leader) {
+        mbar_arrive_expect_tx(bar(C::bQFull + t), C::kQTile);
 #pragma unroll
-      for (int c = 0; c < C::kChunks; ++c)
-        tma_load_3d(sb + C::kQOff + t * C::kQTile + c * C::kQChunk, &p.tm_q, c * 64, U.hq0, tok,
-                    bar(C::bQFull + t));
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_3d(sb + C::kQOff + t * C::kQTile + c * C::kQChunk, &p.tm_q, c * 64, U.hq0, tok,
+                      bar(C::bQFull + t));
+      }
+      __syncwarp();
       ++q_cnt[t];
     }
     for (int n = 0; n < U.nb && ok; ++n) {
       const int tok = U.k_start + U.kv_lo + n * C::BN;
       {
         const uint32_t s = k_cnt % C::KST;
-        ok = mbar_wait(bar(C::bKEmpty + s), ((k_cnt / C::KST) & 1u) ^ 1u, &g_fa_error,
-                       p.timeout_ns);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKEmpty + s), ((k_cnt / C::KST) & 1u) ^ 1u, &g_fa_error,
+                       p.timeout_ns));
         if (!ok) break;
-        mbar_arrive_expect_tx(bar(C::bKFull + s), C::kKVTile);
+        if (leader) {
+          mbar_arrive_expect_tx(bar(C::bKFull + s), C::kKVTile);
 #pragma unroll
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(sb + C::kKOff + s * C::kKVTile + c * C::kKVChunk, &p.tm_k, c * 64, U.hk,
-                      tok, bar(C::bKFull + s));
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d(sb + C::kKOff + s * C::kKVTile + c * C::kKVChunk, &p.tm_k, c * 64, U.hk,
+                        tok, bar(C::bKFull + s));
+        }
+        __syncwarp();
         ++k_cnt;
       }
       {
         const uint32_t s = v_cnt % C::VST;
-        ok = mbar_wait(bar(C::bVEmpty + s), ((v_cnt / C::VST) & 1u) ^ 1u, &g_fa_error,
-                       p.timeout_ns);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bVEmpty + s), ((v_cnt / C::VST) & 1u) ^ 1u, &g_fa_error,
+                       p.timeout_ns));
         if (!ok) break;
-        mbar_arrive_expect_tx(bar(C::bVFull + s), C::kKVTile);
+        if (leader) {
+          mbar_arrive_expect_tx(bar(C::bVFull + s), C::kKVTile);
 #pragma unroll
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(sb + C::kVOff + s * C::kKVTile + c * C::kKVChunk, &p.tm_v, c * 64, U.hk,
-                      tok, bar(C::bVFull + s));
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d(sb + C::kVOff + s * C::kKVTile + c * C::kKVChunk, &p.tm_v, c * 64, U.hk,
+                        tok, bar(C::bVFull + s));
+        }
+        __syncwarp();
         ++v_cnt;
       }
     }
   }
   if (!ok) {
-    // Drain: let every copy this thread issued land before the CTA leaves.
+    // Drain: let every copy this warp issued land before the CTA leaves.
     const uint64_t drain_ns = 200000000ull;
     for (uint32_t i = (k_cnt > C::KST ? k_cnt - C::KST : 0); i < k_cnt; ++i)
       mbar_wait_drain(bar(C::bKFull + i % C::KST), (i / C::KST) & 1u, drain_ns);
@@ -490,7 +504,7 @@ __device__ __forceinline__ void role_producer(const FwdParams &p, uint32_t sb) {
 }
 
 // ---------------------------------------------------------------------------
-// MMA issuer (one thread)
+// MMA issuer (one converged warp; the elected lane issues)
 // ---------------------------------------------------------------------------
 template <class C>
 __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32_t tmem) {
@@ -1103,11 +1117,11 @@ __global__ void __launch_bounds__(C::kThreads, 1) fa_fwd_kernel(const __grid_con
   if (warp < 4) {
     if constexpr (C::kSplitRegs) regs_lower<C::kRegsCtl>();
     if (warp == 0) {
-      if (lane == 0) role_producer<C>(p, sb);
+      role_producer<C>(p, sb);  // whole warp; lane 0 issues the copies
     } else if (warp == 1) {
       role_mma<C>(p, sb, tmem);  // whole warp; MMAs issued by the elected lane
     } else if (warp == 2) {
-      if (lane == 0) role_scheduler<C>(p, sch, sb);
+      role_scheduler<C>(p, sch, sb);  // whole warp; lane 0 publishes
     }
   } else {
     if constexpr (C::kSplitRegs) regs_raise<C::kRegsSoftmax>();
