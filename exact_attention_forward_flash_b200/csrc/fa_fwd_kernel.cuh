@@ -310,10 +310,7 @@ struct FwdCfg {
   static constexpr int kVOff = kKOff + KST * kKVTile;
   // relative-bias staging: one 32-row x 5 x 16-byte buffer per softmax warp,
   // when shared memory allows (otherwise each thread reads its own row)
-  static constexpr int kBiasWarpBytes = 32 * 3 * 16;
-  static constexpr int kBiasOff = kVOff + VST * kKVTile;
-  static constexpr bool kBiasSmem = kBiasOff + NQ * 4 * kBiasWarpBytes + 1024 + 256 <= 232448;
-  static constexpr int kBarOff = kBiasOff + (kBiasSmem ? NQ * 4 * kBiasWarpBytes : 0);
+  static constexpr int kBarOff = kVOff + VST * kKVTile;
   // barrier indices
   static constexpr int bQFull = 0, bQEmpty = NQ, bKFull = 2 * NQ, bKEmpty = bKFull + KST,
                        bVFull = bKEmpty + KST, bVEmpty = bVFull + VST, bSFull = bVEmpty + VST,
@@ -335,7 +332,7 @@ struct FwdCfg {
   // threads = 168 each) is re-split so that the softmax warps hold a whole
   // score row plus the bias staging without spilling.
   static constexpr bool kSplitRegs = NQ == 2;
-  static constexpr uint32_t kRegsCtl = 104, kRegsSoftmax = 200;
+  static constexpr uint32_t kRegsCtl = 72, kRegsSoftmax = 216;
   static_assert(!kSplitRegs || 128 * kRegsCtl + 256 * kRegsSoftmax <= 384 * 168, "register split");
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kOColBase = NQ * NS * BN;
@@ -639,95 +636,59 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
 // ---------------------------------------------------------------------------
 // softmax / correction / epilogue warpgroup (one per Q tile)
 // ---------------------------------------------------------------------------
-// Relative bias of one 16-column chunk for the 32 rows of one warp.
+// Relative bias of one 64-column half of a KV tile, for the calling thread's
+// own row.
 //
-// Row i of the tile needs, for columns c = 16*cc + e (e = 0..15), the bias at
-// distance d = base - c with base = i + (k_len - q_len) - j0.  Those 16 values
-// lie inside the 16-byte-aligned run of 24 values that starts at
-//     a = (base - 16*cc - 15) & ~7,
-// i.e. three 16-byte pieces.  The warp fetches the 32 rows x 3 pieces with
-// lane-contiguous 16-byte loads (piece idx = lane + 32*k belongs to row idx/3;
-// consecutive lanes read consecutive pieces of a row, so a load touches few
-// cache lines), stages them in a per-warp shared buffer, and every thread then
-// reads its own row's three pieces back.  Pieces are either wholly inside
-// [0, rel_extent) or wholly outside (both ends are multiples of 8); those
-// outside are zero.
-constexpr int kBiasPieces = 3;
+// Column c of the half (c = 0..63) sits at distance d = lo + 63 - c from the
+// row's diagonal, where lo is the smallest distance the half meets; its bias
+// is rel_bias[row][d] for 0 <= d < R and 0 elsewhere.  The thread reads the
+// 9 sixteen-byte pieces [a, a + 72) with a = lo rounded down to a multiple of
+// 8, which cover [lo, lo + 63].  R and a are multiples of 8, so a piece lies
+// wholly inside or wholly outside [0, R); pieces outside are not read and
+// count as zero.  The values then sit (lo - a) elements off the word grid
+// and in reverse column order: two select stages shift by whole words and a
+// byte permute per column pair takes the half-word shift and the reversal.
+constexpr int kBiasPieces = 9;
 
-struct BiasFetch {
-  int b0[kBiasPieces];        // distance of column 0 of the unit's first KV tile for the
-                              // row behind each piece (i + k_len - q_len - kv_lo), or a
-                              // sentinel far below zero for rows past the sequence
-  uint32_t off[kBiasPieces];  // offset of that row's bias vector, in 16-byte units
-};
-
-// The bias loads of a tile go out in two batches of NC/2 chunks (one per
-// 64-column half): the first before the thread waits for the tile's scores
-// (their latency hides behind that wait), the second once the first half has
-// taken its bias.  A chunk that no row of the warp meets is neither fetched
-// nor staged.
-template <class C>
-__device__ __forceinline__ unsigned bias_need(const FwdParams &p, int base, bool row_on) {
-  unsigned need = 0;  // warp-uniform: chunks that some row of the warp meets
+__device__ __forceinline__ void bias_fetch(const uint16_t *brow, int lo, int R,
+                                           uint4 (&v)[kBiasPieces]) {
+  const int a = lo & ~7;
+  // one base address (possibly outside the row; only in-range pieces are
+  // dereferenced), pieces at immediate offsets from it
+  const uint4 *src = reinterpret_cast<const uint4 *>(brow) + (a >> 3);
+  const unsigned lim = brow != nullptr ? (unsigned)(R - 8) : 0u;
+  const unsigned ua = brow != nullptr ? (unsigned)a : ~0u;
 #pragma unroll
-  for (int cc = 0; cc < C::BN / 16; ++cc) {
-    const bool nd = row_on && base - 16 * cc >= 0 && base - 16 * cc - 15 < p.R;
-    need |= (__any_sync(0xffffffffu, nd) ? 1u : 0u) << cc;
-  }
-  return need;
+  for (int m = 0; m < kBiasPieces; ++m)
+    v[m] = (ua + 8u * m <= lim) ? ldg_v4(src + m) : make_uint4(0u, 0u, 0u, 0u);
 }
 
-// Issue the loads of chunks [C0, C0 + H) into pf.
-template <class C, int C0>
-__device__ __forceinline__ void bias_load(const FwdParams &p, const BiasFetch &bf, int jrel,
-                                          int lane, unsigned need,
-                                          uint4 (&pf)[4][kBiasPieces]) {
-  constexpr int H = 4;  // chunks of one 64-column half
-#pragma unroll
-  for (int k = 0; k < kBiasPieces; ++k) {
-    const int pc = (lane + 32 * k) % kBiasPieces;  // piece index within the row
-    const int d00 = ((bf.b0[k] - jrel - 15) & ~7) + 8 * pc;
-    const uint4 *rp = reinterpret_cast<const uint4 *>(p.rel_bias) + bf.off[k];
-#pragma unroll
-    for (int h = 0; h < H; ++h) {
-      const int cc = C0 + h;
-      const int d0 = d00 - 16 * cc;  // chunk cc sits 16*cc elements lower
-      const bool in = (need >> cc & 1u) && d0 >= 0 && d0 + 8 <= p.R;
-      pf[h][k] = in ? ldg_v4(rp + (d0 >> 3)) : make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
-}
-
-// Transpose chunk pieces through the warp's buffer and return this row's 16
-// bias values as 16-bit pairs in column order (w2[k]: columns 2k, 2k+1).
-template <class C>
-__device__ __forceinline__ void bias_chunk(uint32_t buf, int lane, int sh,
-                                           const uint4 (&pieces)[kBiasPieces],
-                                           uint32_t (&w2)[8]) {
-  __syncwarp();
-#pragma unroll
-  for (int k = 0; k < kBiasPieces; ++k) sts_v4(buf + (lane + 32 * k) * 16, pieces[k]);
-  __syncwarp();
+// x[c] += bias(c) * inv_scale for the 64 columns of the half (sh = lo & 7).
+template <bool kHalf>
+__device__ __forceinline__ void bias_apply(const uint4 (&v)[kBiasPieces], int sh,
+                                           float inv_scale, float (&x)[64]) {
   uint32_t w[4 * kBiasPieces];
 #pragma unroll
-  for (int k = 0; k < kBiasPieces; ++k) {
-    const uint4 v = lds_v4(buf + (lane * kBiasPieces + k) * 16);
-    w[4 * k] = v.x;
-    w[4 * k + 1] = v.y;
-    w[4 * k + 2] = v.z;
-    w[4 * k + 3] = v.w;
+  for (int m = 0; m < kBiasPieces; ++m) {
+    w[4 * m] = v[m].x;
+    w[4 * m + 1] = v[m].y;
+    w[4 * m + 2] = v[m].z;
+    w[4 * m + 3] = v[m].w;
   }
-  // element q of the aligned run (q = 0..15) is the value at distance
-  // base - 16*cc - 15 + q, i.e. column 15 - q of the chunk
-  const int sw = sh >> 1;
+  const int sw = sh >> 1;  // whole-word shift, 0..3
 #pragma unroll
-  for (int k = 0; k < 10; ++k) w[k] = (sw & 2) ? w[k + 2] : w[k];
+  for (int j = 0; j < 34; ++j) w[j] = (sw & 2) ? w[j + 2] : w[j];
 #pragma unroll
-  for (int k = 0; k < 9; ++k) w[k] = (sw & 1) ? w[k + 1] : w[k];
-  // pick two consecutive aligned elements, swapped into column order
+  for (int j = 0; j < 33; ++j) w[j] = (sw & 1) ? w[j + 1] : w[j];
+  // column pair (2k, 2k+1) -> low / high half of one word
   const uint32_t sel = (sh & 1) ? 0x3254u : 0x1032u;
+  const uint64_t isc = f2(inv_scale, inv_scale);
 #pragma unroll
-  for (int e2 = 0; e2 < 8; ++e2) w2[7 - e2] = __byte_perm(w[e2], w[e2 + 1], sel);
+  for (int k = 0; k < 32; ++k) {
+    const uint32_t pw = __byte_perm(w[31 - k], w[32 - k], sel);
+    f2_split(ffma2(f2(lo_f<kHalf>(pw), hi_f<kHalf>(pw)), isc, f2(x[2 * k], x[2 * k + 1])),
+             x[2 * k], x[2 * k + 1]);
+  }
 }
 
 template <class C>
@@ -738,7 +699,6 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
   const int tid = static_cast<int>(threadIdx.x) - 128 * (t + 1);  // tile row == TMEM lane
   const int lane = tid & 31;
   const uint32_t lane_addr = static_cast<uint32_t>(tid & ~31) << 16;
-  const uint32_t bias_buf = sb + C::kBiasOff + (t * 4 + (tid >> 5)) * C::kBiasWarpBytes;
   const float sl2 = p.scale_log2;
   uint32_t s_cnt = 0;
   bool ok = true;
@@ -773,22 +733,6 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
     const bool has_bias = p.rel_bias != nullptr;
     const uint16_t *brow = nullptr;
     if (has_bias && valid) brow = p.rel_bias + orow * p.R;
-    BiasFetch bf;
-    if constexpr (C::kBiasSmem) {
-      if (has_bias) {
-#pragma unroll
-        for (int kk = 0; kk < kBiasPieces; ++kk) {
-          const int idx = lane + 32 * kk;
-          const int rr = U.row0 + t * kBM + (tid & ~31) + idx / kBiasPieces;
-          const int ii = rr >> p.lgP;
-          const int hh = U.hq0 + (rr & (p.P - 1));
-          const bool v = ii < U.q_len;
-          bf.b0[kk] = v ? ii + U.delta - U.kv_lo : -(1 << 30);
-          bf.off[kk] = v ? (uint32_t)((((size_t)(U.q_start + ii) * p.Hq + hh) * p.R) >> 3) : 0u;
-        }
-      }
-    }
-
     float m_ref = -INFINITY, l = 0.f;
     for (int n = 0; n < nb; ++n) {
       const uint32_t g = s_cnt + n;
@@ -835,67 +779,51 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
         };
       // The two kinds of tile take disjoint paths (each with its own wait) so
       // that their register-resident arrays never meet at a join.
-      if (C::kBiasSmem && bias_blk) {
-        const unsigned need = bias_need<C>(p, base, valid);
-        uint4 pf[4][kBiasPieces];  // bias pieces of one 64-column half
-        bias_load<C, 0>(p, bf, jrel, lane, need, pf);  // in flight during the wait
+      if (bias_blk) {
+        // Tiles that meet the bias band: 64-column halves, each with its own
+        // running-max update (online softmax at half-tile granularity), so
+        // that a half's bias and its scores fit in registers together.  With
+        // conditional rescaling the second half rarely moves the reference
+        // max; when it does, the first half's P (already in tensor memory) is
+        // rescaled along with O and l.  A half's bias loads are in flight
+        // while the thread waits for the scores (first half) or works on the
+        // half before it.
+        const int lo0 = base - 63;  // smallest distance met by half 0
+        const int bsh = lo0 & 7;    // misalignment, the same for every half of the row
+        auto half_on = [&](int lo) {  // some row of the warp meets the band in this half
+          return __any_sync(0xffffffffu, brow != nullptr && lo + 63 >= 0 && lo < p.R);
+        };
+        uint4 bv[kBiasPieces];
+        bool bon = half_on(lo0);
+        if (bon) bias_fetch(brow, lo0, p.R, bv);
         ok = wait_scores();
         if (!ok) break;
         if (warp_on) {
-          // Tiles that meet the bias band: 64-column halves, each with its own
-          // running-max update (online softmax at half-tile granularity), so
-          // that the staged bias and the scores fit in registers together.
-          // With conditional rescaling the second half rarely moves the
-          // reference max; when it does, the first half's P (already in tensor
-          // memory) is rescaled along with O and l.
-          const bool staged = true;
 #pragma unroll
-        for (int hf = 0; hf < BN / 64; ++hf) {
-          float x[64];
-          {
-            uint32_t r0[32], r1[32];
-            tmem_ld32(s_addr + 64 * hf, r0);
-            tmem_ld32(s_addr + 64 * hf + 32, r1);
-            tmem_wait_ld();
+          for (int hf = 0; hf < BN / 64; ++hf) {
+            float x[64];
+            {
+              uint32_t r0[32], r1[32];
+              tmem_ld32(s_addr + 64 * hf, r0);
+              tmem_ld32(s_addr + 64 * hf + 32, r1);
+              tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              x[e] = __uint_as_float(r0[e]);
-              x[32 + e] = __uint_as_float(r1[e]);
-            }
-          }
-          if constexpr (C::kBiasSmem) {
-            if (staged) {
-              const int sh = (base - 15) & 7;  // misalignment of the bias run
-              const uint64_t isc = f2(p.inv_scale, p.inv_scale);
-#pragma unroll
-              for (int cc = 0; cc < 4; ++cc) {
-                if (need >> (4 * hf + cc) & 1u) {
-                  uint32_t w2[8];
-                  bias_chunk<C>(bias_buf, lane, sh, pf[cc], w2);
-#pragma unroll
-                  for (int e = 0; e < 8; ++e)
-                    f2_split(ffma2(f2(lo_f<C::HALF>(w2[e]), hi_f<C::HALF>(w2[e])), isc,
-                                   f2(x[16 * cc + 2 * e], x[16 * cc + 2 * e + 1])),
-                             x[16 * cc + 2 * e], x[16 * cc + 2 * e + 1]);
-                }
-              }
-              if (hf + 1 < BN / 64) bias_load<C, 4>(p, bf, jrel, lane, need, pf);
-            }
-          } else {
-            // relative bias without shared staging: column c at distance base - c
-            if (brow != nullptr) {
-#pragma unroll
-              for (int e = 0; e < 64; ++e) {
-                const int d = base - (64 * hf + e);
-                if (d >= 0 && d < p.R) x[e] += load_elem<C::HALF>(brow + d) * p.inv_scale;
+              for (int e = 0; e < 32; ++e) {
+                x[e] = __uint_as_float(r0[e]);
+                x[32 + e] = __uint_as_float(r1[e]);
               }
             }
-          }
-          if (lim_c < 64 * hf + 64) {
+            if (bon) bias_apply<C::HALF>(bv, bsh, p.inv_scale, x);
+            if (hf + 1 < BN / 64) {
+              const int lo = lo0 - 64 * (hf + 1);
+              bon = half_on(lo);
+              if (bon) bias_fetch(brow, lo, p.R, bv);
+            }
+            if (lim_c < 64 * hf + 64) {
 #pragma unroll
-            for (int e = 0; e < 64; ++e)
-              if (64 * hf + e >= lim_c) x[e] = -INFINITY;
-          }
+              for (int e = 0; e < 64; ++e)
+                if (64 * hf + e >= lim_c) x[e] = -INFINITY;
+            }
           // running-max update with conditional rescaling
           const float m_new = fmaxf(m_ref, row_max<0, 64>(x));
           if (n == 0 && hf == 0) {
@@ -936,7 +864,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
           // P half hf -> columns [32 hf, 32 hf + 32): only score columns
           // already read are overwritten
           tmem_st32(s_addr + 32 * hf, pk);
-        }
+          }
           if (!ok) break;
           tmem_wait_st();
         }
@@ -958,16 +886,6 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
             for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(r[e]);
           }
           tmem_wait_ld();
-          if constexpr (!C::kBiasSmem) {
-            // relative bias without shared staging: column c at distance base - c
-            if (brow != nullptr && base >= 0 && base - (BN - 1) < p.R) {
-#pragma unroll
-              for (int c = 0; c < BN; ++c) {
-                const int d = base - c;
-                if (d >= 0 && d < p.R) s[c] += load_elem<C::HALF>(brow + d) * p.inv_scale;
-              }
-            }
-          }
           if (lim_c < BN) {
 #pragma unroll
             for (int c = 0; c < BN; ++c)
