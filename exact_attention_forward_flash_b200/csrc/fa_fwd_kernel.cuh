@@ -308,14 +308,22 @@ struct FwdCfg {
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + NQ * kQTile;
   static constexpr int kVOff = kKOff + KST * kKVTile;
-  // relative-bias staging: one 32-row x 5 x 16-byte buffer per softmax warp,
-  // when shared memory allows (otherwise each thread reads its own row)
   static constexpr int kBarOff = kVOff + VST * kKVTile;
+  // Split P.V (single S buffer, 128-key tiles): P.V starts on the first 64
+  // keys once the softmax has stored their half of P, overlapping the second
+  // half's exponentials; the rest follows the whole of P.
+  static constexpr bool kSplitPV = NS == 1 && BN == 128;
+  // Split score MMA as well: P(n) fills columns [0, 64) of its tile's S
+  // buffer, so the keys 64..127 of S(n+1), which land in columns [64, 128),
+  // can be computed as soon as the softmax has read S(n).  Measured slower:
+  // 128x64 MMAs issue at ~50 cycles for 32 of work.
+  static constexpr bool kSplitS = false;
   // barrier indices
   static constexpr int bQFull = 0, bQEmpty = NQ, bKFull = 2 * NQ, bKEmpty = bKFull + KST,
                        bVFull = bKEmpty + KST, bVEmpty = bVFull + VST, bSFull = bVEmpty + VST,
                        bPFull = bSFull + NQ * NS, bOFull = bPFull + NQ * NS,
-                       bOEmpty = bOFull + NQ * NS, bDrain = bOEmpty + NQ,
+                       bOEmpty = bOFull + NQ * NS, bSRead = bOEmpty + NQ, bPHalf = bSRead + NQ,
+                       bDrain = bPHalf + NQ,
                        bUFull = bDrain + 1, bUEmpty = bUFull + kUnitRing,
                        kNumBars = bUEmpty + kUnitRing;
   // consumers of each published unit: producer, MMA issuer, every softmax warp
@@ -330,7 +338,7 @@ struct FwdCfg {
   static constexpr int kThreads = 128 * (1 + NQ);
   // registers: with two softmax warpgroups the launch budget (65536 / 384
   // threads = 168 each) is re-split so that the softmax warps hold a whole
-  // score row plus the bias staging without spilling.
+  // score row, or half a row plus its bias window, without spilling.
   static constexpr bool kSplitRegs = NQ == 2;
   static constexpr uint32_t kRegsCtl = 72, kRegsSoftmax = 216;
   static_assert(!kSplitRegs || 128 * kRegsCtl + 256 * kRegsSoftmax <= 384 * 168, "register split");
@@ -543,6 +551,33 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
     tc_commit_elect(bar(C::bOFull + t * C::NS + g % C::NS));
   };
 
+  // split form: keys [64 hi, 64 hi + 64) of S_t into columns [64 hi, 64 hi + 64)
+  constexpr uint32_t idesc_s64 = instr_desc<C::HALF>(kBM, 64, false, false);
+  auto issue_s_half = [&](int t, uint32_t g, uint32_t kstage, int hi) {
+    const uint32_t qa = sb + C::kQOff + t * C::kQTile;
+    const uint32_t ka = sb + C::kKOff + kstage * C::kKVTile + hi * 64 * 128;
+    const uint32_t d_tmem = tmem + C::s_col(t, g % C::NS) + hi * 64;
+#pragma unroll
+    for (int kk = 0; kk < C::D / 16; ++kk) {
+      const uint32_t off = (kk % 4) * 32;
+      const uint64_t a = smem_desc_sw128(qa + (kk / 4) * C::kQChunk + off, 16, 1024);
+      const uint64_t b = smem_desc_sw128(ka + (kk / 4) * C::kKVChunk + off, 16, 1024);
+      tc_mma_ss_elect(d_tmem, a, b, idesc_s64, kk > 0 ? 1u : 0u);
+    }
+  };
+  // split form: O_t += P_t[:, 64 hi .. 64 hi + 64) V[64 hi .. 64 hi + 64, :]
+  auto issue_pv_half = [&](int t, uint32_t g, uint32_t vstage, bool first, int hi) {
+    const uint32_t va = sb + C::kVOff + vstage * C::kKVTile;
+    const uint32_t p_tmem = tmem + C::s_col(t, g % C::NS);
+    const uint32_t d_tmem = tmem + C::o_col(t);
+#pragma unroll
+    for (int k4 = 0; k4 < 4; ++k4) {
+      const int kk = 4 * hi + k4;
+      const uint64_t b = smem_desc_sw128(va + kk * 16 * 128, C::kKVChunk, 1024);
+      tc_mma_ts_elect(d_tmem, p_tmem + kk * 8, b, idesc_pv, (first && kk == 0) ? 0u : 1u);
+    }
+  };
+
   uint32_t ucnt = 0;
   Unit U;
   while (ok && next_unit<C>(p, sb, ucnt, U, ok, true)) {
@@ -589,6 +624,7 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
         tc_commit_elect(bar(C::bKEmpty + kn % C::KST));
       }
       const uint32_t vn = vb + n;
+      bool k_next_ready = false;  // K tile n+1 waited for (split form)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bVFull + vn % C::VST), (vn / C::VST) & 1u, &g_fa_error,
                      p.timeout_ns));
       if (!ok) break;
@@ -599,6 +635,55 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
         if (n == 0) {
           ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bOEmpty + t), (u_cnt[t] & 1u) ^ 1u, &g_fa_error, p.timeout_ns));
           if (!ok) break;
+        }
+        if constexpr (C::kSplitPV) {
+          // keys 64..127 of S_t(n+1) as soon as S_t(n) has been read (split S); P.V on
+          // the first 64 keys once their half of P is stored, then the rest;
+          // keys 0..63 of S_t(n+1) after P.V has read P_t(n)
+          const bool more = n + 1 < nb;
+          if (C::kSplitS && more) {
+            if (!k_next_ready) {
+              ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + kn % C::KST),
+                                                     (kn / C::KST) & 1u, &g_fa_error, p.timeout_ns));
+              if (!ok) break;
+              k_next_ready = true;
+            }
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bSRead + t), g & 1u, &g_fa_error,
+                                                   p.timeout_ns));
+            if (!ok) break;
+            tc_fence_after();
+            issue_s_half(t, g + 1, kn % C::KST, 1);
+          }
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bPHalf + t), g & 1u, &g_fa_error,
+                                                 p.timeout_ns));
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv_half(t, g, vn % C::VST, n == 0, 0);
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bPFull + t), g & 1u, &g_fa_error,
+                                                 p.timeout_ns));
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv_half(t, g, vn % C::VST, n == 0, 1);
+          tc_commit_elect(bar(C::bOFull + t));
+          if (t == last_t) tc_commit_elect(bar(C::bVEmpty + vn % C::VST));
+          if (more) {
+            if (C::kSplitS) {
+              issue_s_half(t, g + 1, kn % C::KST, 0);
+              tc_commit_elect(bar(C::bSFull + t));
+            } else {
+              if (!k_next_ready) {
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + kn % C::KST),
+                                                       (kn / C::KST) & 1u, &g_fa_error, p.timeout_ns));
+                if (!ok) break;
+                tc_fence_after();
+                k_next_ready = true;
+              }
+              issue_s(t, g + 1, kn % C::KST);  // commits the S barrier itself
+            }
+            if (n + 1 == nb - 1) tc_commit_elect(bar(C::bQEmpty + t));
+            if (t == last_t) tc_commit_elect(bar(C::bKEmpty + kn % C::KST));
+          }
+          continue;
         }
         ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bPFull + t * C::NS + g % C::NS), (g / C::NS) & 1u, &g_fa_error,
                        p.timeout_ns));
@@ -747,6 +832,12 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
       // no row of the warp has a masked column here: the FMA-pipe exponential
       // may stand in for some of the MUFU ones
       const bool poly_ok = __all_sync(0xffffffffu, lim_c >= BN);
+      // one arrival per warp, after this thread's tensor-memory accesses
+      auto warp_arrive = [&](int b) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(b));
+      };
       auto wait_scores = [&]() -> bool {
         const bool w = __all_sync(0xffffffffu,
                                   mbar_wait(bar(C::bSFull + t * NS + buf), (g / NS) & 1u,
@@ -813,6 +904,8 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
                 x[32 + e] = __uint_as_float(r1[e]);
               }
             }
+            // every score read: the next tile's upper keys may land
+            if (C::kSplitS && hf == BN / 64 - 1) warp_arrive(C::bSRead + t);
             if (bon) bias_apply<C::HALF>(bv, bsh, p.inv_scale, x);
             if (hf + 1 < BN / 64) {
               const int lo = lo0 - 64 * (hf + 1);
@@ -867,10 +960,13 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
           }
           if (!ok) break;
           tmem_wait_st();
+        } else if (C::kSplitS) {
+          warp_arrive(C::bSRead + t);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(C::bPFull + t * NS + buf));
+        // the bias path may rescale its first P half after storing it, so the
+        // first-half signal waits for the whole tile
+        if (C::kSplitPV) warp_arrive(C::bPHalf + t);
+        warp_arrive(C::bPFull + t * NS + buf);
       } else {
         ok = wait_scores();
         if (!ok) break;
@@ -886,6 +982,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
             for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(r[e]);
           }
           tmem_wait_ld();
+          if (C::kSplitS) warp_arrive(C::bSRead + t);
           if (lim_c < BN) {
 #pragma unroll
             for (int c = 0; c < BN; ++c)
@@ -915,6 +1012,10 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
             else
               l += exp_pack<C::HALF, false, 0, 64>(s, sl2, mc, pk);
             tmem_st32(s_addr, pk);
+            if (C::kSplitPV) {
+              tmem_wait_st();
+              warp_arrive(C::bPHalf + t);
+            }
           }
           if constexpr (BN == 128) {
             uint32_t pk[32];
@@ -925,13 +1026,11 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
             tmem_st32(s_addr + 32, pk);
           }
           tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(C::bPFull + t * NS + buf));
+          warp_arrive(C::bPFull + t * NS + buf);
         } else {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(C::bPFull + t * NS + buf));
+          if (C::kSplitS) warp_arrive(C::bSRead + t);
+          if (C::kSplitPV) warp_arrive(C::bPHalf + t);
+          warp_arrive(C::bPFull + t * NS + buf);
         }
       }
     }
@@ -1005,6 +1104,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) fa_fwd_kernel(const __grid_con
     for (int b = 0; b < C::kNumBars; ++b) {
       uint32_t cnt = 1;
       if (b >= C::bPFull && b < C::bPFull + C::NQ * C::NS) cnt = 4;  // one per warp
+      if (b >= C::bSRead && b < C::bPHalf + C::NQ) cnt = 4;
       if (b >= C::bOEmpty && b < C::bOEmpty + C::NQ) cnt = 128;
       if (b >= C::bUEmpty && b < C::bUEmpty + kUnitRing) cnt = C::kUnitConsumers;
       mbar_init(sb + C::kBarOff + 8u * b, cnt);
