@@ -128,8 +128,8 @@ int num_sms(int dev) {
 }
 
 // kernel variants
-using Fwd128B = FwdCfg<128, 128, 2, 1, 2, 2, false, false>;
-using Fwd128H = FwdCfg<128, 128, 2, 1, 2, 2, true, false>;
+using Fwd128B = FwdCfg<128, 128, 2, 1, 3, 0, false, false>;
+using Fwd128H = FwdCfg<128, 128, 2, 1, 3, 0, true, false>;
 using Fwd256B = FwdCfg<256, 64, 1, 2, 3, 2, false, false>;
 using Fwd256H = FwdCfg<256, 64, 1, 2, 3, 2, true, false>;
 using Spl128B = FwdCfg<128, 128, 1, 2, 3, 3, false, true>;

@@ -17,8 +17,9 @@
 //               publishes them, one record each, through a small ring in
 //               shared memory that the other roles read in the same order.
 //   warp 0      TMA producer: Q tiles once per unit, then K and V tiles of
-//               BN keys through separate KST-/VST-stage shared-memory rings.
-//   warp 1      MMA issuer (one thread): S = Q K^T (SS form, both operands
+//               BN keys through shared-memory rings (separate K and V rings,
+//               or one ring that K and V tiles take in turn).
+//   warp 1      MMA issuer (the warp's elected lane): S = Q K^T (SS form, both operands
 //               K-major in 128B-swizzled shared memory) into tensor memory,
 //               and O += P V (TS form: P read from tensor memory where it
 //               overwrites S, V MN-major in shared memory).  Also owns the
@@ -306,9 +307,13 @@ struct FwdCfg {
   static constexpr int kQChunk = kBM * 128;       // bytes of one 64-column chunk
   static constexpr int kKVChunk = BN * 128;
   static constexpr int kQOff = 0;
+  // K/V stages: separate rings of KST and VST slots, or (VST == 0) one ring of
+  // KST slots that the K and V tiles take in turn -- K(n), V(n), K(n+1), ...
+  // -- so that K(n+1) reuses the slot of V(n-1) and V(n+1) that of K(n).
+  static constexpr bool kKVRing = VST == 0;
   static constexpr int kKOff = kQOff + NQ * kQTile;
-  static constexpr int kVOff = kKOff + KST * kKVTile;
-  static constexpr int kBarOff = kVOff + VST * kKVTile;
+  static constexpr int kVOff = kKVRing ? kKOff : kKOff + KST * kKVTile;
+  static constexpr int kBarOff = kKOff + (KST + VST) * kKVTile;
   // Split P.V (single S buffer, 128-key tiles): P.V starts on the first 64
   // keys once the softmax has stored their half of P, overlapping the second
   // half's exponentials; the rest follows the whole of P.
@@ -320,7 +325,8 @@ struct FwdCfg {
   static constexpr bool kSplitS = false;
   // barrier indices
   static constexpr int bQFull = 0, bQEmpty = NQ, bKFull = 2 * NQ, bKEmpty = bKFull + KST,
-                       bVFull = bKEmpty + KST, bVEmpty = bVFull + VST, bSFull = bVEmpty + VST,
+                       bVFull0 = bKEmpty + KST, bVEmpty0 = bVFull0 + VST, bSFull = bVEmpty0 + VST,
+                       bVFull = kKVRing ? bKFull : bVFull0, bVEmpty = kKVRing ? bKEmpty : bVEmpty0,
                        bPFull = bSFull + NQ * NS, bOFull = bPFull + NQ * NS,
                        bOEmpty = bOFull + NQ * NS, bSRead = bOEmpty + NQ, bPHalf = bSRead + NQ,
                        bDrain = bPHalf + NQ,
@@ -347,6 +353,20 @@ struct FwdCfg {
   static_assert(kOColBase + NQ * D <= 512, "tensor memory budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(D % 64 == 0 && BN % 32 == 0 && (BN == 64 || BN == 128), "tile shape");
+  // slot and phase parity of the K tile k / V tile v (counted over the CTA's
+  // whole sequence of KV tiles), and the barriers of V slots
+  __host__ __device__ static constexpr uint32_t k_slot(uint32_t k) {
+    return kKVRing ? (2u * k) % KST : k % KST;
+  }
+  __host__ __device__ static constexpr uint32_t k_par(uint32_t k) {
+    return kKVRing ? ((2u * k) / KST) & 1u : (k / KST) & 1u;
+  }
+  __host__ __device__ static constexpr uint32_t v_slot(uint32_t v) {
+    return kKVRing ? (2u * v + 1u) % KST : v % VST;
+  }
+  __host__ __device__ static constexpr uint32_t v_par(uint32_t v) {
+    return kKVRing ? ((2u * v + 1u) / KST) & 1u : (v / VST) & 1u;
+  }
   __host__ __device__ static constexpr int s_col(int t, int b) { return (t * NS + b) * BN; }
   __host__ __device__ static constexpr int o_col(int t) { return kOColBase + t * D; }
 };
@@ -464,8 +484,8 @@ __device__ __forceinline__ void role_producer(const FwdParams &p, uint32_t sb) {
     for (int n = 0; n < U.nb && ok; ++n) {
       const int tok = U.k_start + U.kv_lo + n * C::BN;
       {
-        const uint32_t s = k_cnt % C::KST;
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKEmpty + s), ((k_cnt / C::KST) & 1u) ^ 1u, &g_fa_error,
+        const uint32_t s = C::k_slot(k_cnt);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKEmpty + s), C::k_par(k_cnt) ^ 1u, &g_fa_error,
                        p.timeout_ns));
         if (!ok) break;
         if (leader) {
@@ -479,8 +499,8 @@ __device__ __forceinline__ void role_producer(const FwdParams &p, uint32_t sb) {
         ++k_cnt;
       }
       {
-        const uint32_t s = v_cnt % C::VST;
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bVEmpty + s), ((v_cnt / C::VST) & 1u) ^ 1u, &g_fa_error,
+        const uint32_t s = C::v_slot(v_cnt);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bVEmpty + s), C::v_par(v_cnt) ^ 1u, &g_fa_error,
                        p.timeout_ns));
         if (!ok) break;
         if (leader) {
@@ -498,10 +518,17 @@ __device__ __forceinline__ void role_producer(const FwdParams &p, uint32_t sb) {
   if (!ok) {
     // Drain: let every copy this warp issued land before the CTA leaves.
     const uint64_t drain_ns = 200000000ull;
-    for (uint32_t i = (k_cnt > C::KST ? k_cnt - C::KST : 0); i < k_cnt; ++i)
-      mbar_wait_drain(bar(C::bKFull + i % C::KST), (i / C::KST) & 1u, drain_ns);
-    for (uint32_t i = (v_cnt > C::VST ? v_cnt - C::VST : 0); i < v_cnt; ++i)
-      mbar_wait_drain(bar(C::bVFull + i % C::VST), (i / C::VST) & 1u, drain_ns);
+    // the latest load of every slot
+    if constexpr (C::kKVRing) {
+      const uint32_t n_items = k_cnt + v_cnt;  // K and V tiles issued, in ring order
+      for (uint32_t it = (n_items > C::KST ? n_items - C::KST : 0); it < n_items; ++it)
+        mbar_wait_drain(bar(C::bKFull + it % C::KST), (it / C::KST) & 1u, drain_ns);
+    } else {
+      for (uint32_t i = (k_cnt > C::KST ? k_cnt - C::KST : 0); i < k_cnt; ++i)
+        mbar_wait_drain(bar(C::bKFull + C::k_slot(i)), C::k_par(i), drain_ns);
+      for (uint32_t i = (v_cnt > C::VST ? v_cnt - C::VST : 0); i < v_cnt; ++i)
+        mbar_wait_drain(bar(C::bVFull + C::v_slot(i)), C::v_par(i), drain_ns);
+    }
 #pragma unroll
     for (int t = 0; t < C::NQ; ++t)
       if (q_cnt[t]) mbar_wait_drain(bar(C::bQFull + t), (q_cnt[t] - 1) & 1u, drain_ns);
@@ -597,35 +624,35 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
     const uint32_t kb = k_cnt, vb = v_cnt;
 
     // prologue: S(0) for every active tile
-    ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + kb % C::KST), (kb / C::KST) & 1u, &g_fa_error, p.timeout_ns));
+    ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + C::k_slot(kb)), C::k_par(kb), &g_fa_error, p.timeout_ns));
     if (!ok) break;
     tc_fence_after();
 #pragma unroll
     for (int t = 0; t < C::NQ; ++t) {
       if (!(U.active >> t & 1u)) continue;
-      issue_s(t, sbase[t], kb % C::KST);
+      issue_s(t, sbase[t], C::k_slot(kb));
       if (nb == 1) tc_commit_elect(bar(C::bQEmpty + t));
     }
-    tc_commit_elect(bar(C::bKEmpty + kb % C::KST));
+    tc_commit_elect(bar(C::bKEmpty + C::k_slot(kb)));
 
     for (int n = 0; n < nb && ok; ++n) {
       const uint32_t kn = kb + n + 1;  // K tile of block n+1
       if (C::NS == 2 && n + 1 < nb) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + kn % C::KST), (kn / C::KST) & 1u, &g_fa_error,
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + C::k_slot(kn)), C::k_par(kn), &g_fa_error,
                        p.timeout_ns));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
         for (int t = 0; t < C::NQ; ++t) {
           if (!(U.active >> t & 1u)) continue;
-          issue_s(t, sbase[t] + n + 1, kn % C::KST);
+          issue_s(t, sbase[t] + n + 1, C::k_slot(kn));
           if (n + 1 == nb - 1) tc_commit_elect(bar(C::bQEmpty + t));
         }
-        tc_commit_elect(bar(C::bKEmpty + kn % C::KST));
+        tc_commit_elect(bar(C::bKEmpty + C::k_slot(kn)));
       }
       const uint32_t vn = vb + n;
       bool k_next_ready = false;  // K tile n+1 waited for (split form)
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bVFull + vn % C::VST), (vn / C::VST) & 1u, &g_fa_error,
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bVFull + C::v_slot(vn)), C::v_par(vn), &g_fa_error,
                      p.timeout_ns));
       if (!ok) break;
 #pragma unroll
@@ -643,8 +670,8 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
           const bool more = n + 1 < nb;
           if (C::kSplitS && more) {
             if (!k_next_ready) {
-              ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + kn % C::KST),
-                                                     (kn / C::KST) & 1u, &g_fa_error, p.timeout_ns));
+              ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + C::k_slot(kn)),
+                                                     C::k_par(kn), &g_fa_error, p.timeout_ns));
               if (!ok) break;
               k_next_ready = true;
             }
@@ -652,36 +679,36 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
                                                    p.timeout_ns));
             if (!ok) break;
             tc_fence_after();
-            issue_s_half(t, g + 1, kn % C::KST, 1);
+            issue_s_half(t, g + 1, C::k_slot(kn), 1);
           }
           ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bPHalf + t), g & 1u, &g_fa_error,
                                                  p.timeout_ns));
           if (!ok) break;
           tc_fence_after();
-          issue_pv_half(t, g, vn % C::VST, n == 0, 0);
+          issue_pv_half(t, g, C::v_slot(vn), n == 0, 0);
           ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bPFull + t), g & 1u, &g_fa_error,
                                                  p.timeout_ns));
           if (!ok) break;
           tc_fence_after();
-          issue_pv_half(t, g, vn % C::VST, n == 0, 1);
+          issue_pv_half(t, g, C::v_slot(vn), n == 0, 1);
           tc_commit_elect(bar(C::bOFull + t));
-          if (t == last_t) tc_commit_elect(bar(C::bVEmpty + vn % C::VST));
+          if (t == last_t) tc_commit_elect(bar(C::bVEmpty + C::v_slot(vn)));
           if (more) {
             if (C::kSplitS) {
-              issue_s_half(t, g + 1, kn % C::KST, 0);
+              issue_s_half(t, g + 1, C::k_slot(kn), 0);
               tc_commit_elect(bar(C::bSFull + t));
             } else {
               if (!k_next_ready) {
-                ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + kn % C::KST),
-                                                       (kn / C::KST) & 1u, &g_fa_error, p.timeout_ns));
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + C::k_slot(kn)),
+                                                       C::k_par(kn), &g_fa_error, p.timeout_ns));
                 if (!ok) break;
                 tc_fence_after();
                 k_next_ready = true;
               }
-              issue_s(t, g + 1, kn % C::KST);  // commits the S barrier itself
+              issue_s(t, g + 1, C::k_slot(kn));  // commits the S barrier itself
             }
             if (n + 1 == nb - 1) tc_commit_elect(bar(C::bQEmpty + t));
-            if (t == last_t) tc_commit_elect(bar(C::bKEmpty + kn % C::KST));
+            if (t == last_t) tc_commit_elect(bar(C::bKEmpty + C::k_slot(kn)));
           }
           continue;
         }
@@ -689,18 +716,18 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
                        p.timeout_ns));
         if (!ok) break;
         tc_fence_after();
-        issue_pv(t, g, vn % C::VST, n == 0);
-        if (t == last_t) tc_commit_elect(bar(C::bVEmpty + vn % C::VST));
+        issue_pv(t, g, C::v_slot(vn), n == 0);
+        if (t == last_t) tc_commit_elect(bar(C::bVEmpty + C::v_slot(vn)));
         if (C::NS == 1 && n + 1 < nb) {
           if (t == 0) {
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + kn % C::KST), (kn / C::KST) & 1u, &g_fa_error,
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + C::k_slot(kn)), C::k_par(kn), &g_fa_error,
                            p.timeout_ns));
             if (!ok) break;
             tc_fence_after();
           }
-          issue_s(t, g + 1, kn % C::KST);
+          issue_s(t, g + 1, C::k_slot(kn));
           if (n + 1 == nb - 1) tc_commit_elect(bar(C::bQEmpty + t));
-          if (t == last_t) tc_commit_elect(bar(C::bKEmpty + kn % C::KST));
+          if (t == last_t) tc_commit_elect(bar(C::bKEmpty + C::k_slot(kn)));
         }
       }
     }
