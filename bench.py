@@ -36,13 +36,14 @@ if ROOT not in sys.path:
 
 METRIC = "attention fwd TFLOP/s & % of BF16 tensor peak; split-KV decode HBM GB/s"
 MAIN = "varlen_gqa_bias"
-EXTRAS = ["dense_257", "video_dit_20480", "encoder_d256_seqused", "decode_splitkv"]
+EXTRAS = ["dense_257", "video_dit_20480", "encoder_d256_seqused", "decode_splitkv", "dense_d64"]
 DESCR = {
     "dense_257": "dense non-causal MHA B=1 S=257 H=8 D=128 bf16",
     "varlen_gqa_bias": "varlen causal GQA 32/8 D=128, 4 seqs U[512,4096] (seeded), rel_bias R=256 bf16",
     "video_dit_20480": "dense non-causal MHA B=1 S=20480 H=56 D=128 bf16",
     "encoder_d256_seqused": "dense GQA 8/1 D=256 B=2 Sq=1024 Sk=1024 seqused_k=968 bf16",
     "decode_splitkv": "split-KV decode B=8 Sq=1 Sk=131072 Hq=32 Hkv=8 D=128 bf16",
+    "dense_d64": "dense non-causal MHA B=4 S=4096 H=16 D=64 bf16",
 }
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
 

@@ -128,10 +128,14 @@ int num_sms(int dev) {
 }
 
 // kernel variants
+using Fwd64B = FwdCfg<64, 128, 2, 1, 3, 0, false, false>;
+using Fwd64H = FwdCfg<64, 128, 2, 1, 3, 0, true, false>;
 using Fwd128B = FwdCfg<128, 128, 2, 1, 3, 0, false, false>;
 using Fwd128H = FwdCfg<128, 128, 2, 1, 3, 0, true, false>;
 using Fwd256B = FwdCfg<256, 64, 1, 2, 3, 2, false, false>;
 using Fwd256H = FwdCfg<256, 64, 1, 2, 3, 2, true, false>;
+using Spl64B = FwdCfg<64, 128, 1, 2, 3, 3, false, true>;
+using Spl64H = FwdCfg<64, 128, 1, 2, 3, 3, true, true>;
 using Spl128B = FwdCfg<128, 128, 1, 2, 3, 3, false, true>;
 using Spl128H = FwdCfg<128, 128, 1, 2, 3, 3, true, true>;
 using Spl256B = FwdCfg<256, 64, 1, 2, 2, 2, false, true>;
@@ -179,8 +183,8 @@ fa_status validate(const Common &c) {
   if (c.B < 0 || c.Hq <= 0 || c.Hkv <= 0 || c.D <= 0)
     return fail(FA_ERR_INVALID, "B must be >= 0 and Hq, Hkv, D > 0");
   if (c.Hq % c.Hkv != 0) return fail(FA_ERR_INVALID, "Hq (%d) must be a multiple of Hkv (%d)", c.Hq, c.Hkv);
-  if (c.D != 128 && c.D != 256)
-    return fail(FA_ERR_UNSUPPORTED, "head_dim %d not served (128 or 256)", c.D);
+  if (c.D != 64 && c.D != 128 && c.D != 256)
+    return fail(FA_ERR_UNSUPPORTED, "head_dim %d not served (64, 128 or 256)", c.D);
   if (!c.varlen && (c.Sq < 0 || c.Sk < 0)) return fail(FA_ERR_INVALID, "Sq, Sk must be >= 0");
   if (c.varlen && (c.total_q < 0 || c.total_k < 0 || c.max_q < 0))
     return fail(FA_ERR_INVALID, "total_q, total_k, max_seqlen_q must be >= 0");
@@ -276,10 +280,12 @@ fa_status run_fwd(const Common &c, cudaStream_t st) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return fail(FA_ERR_CUDA, "cudaGetDevice failed");
   FwdParams p;
-  if ((s = fill_params(c, p, c.D == 128 ? 2 : 1, c.D == 128 ? 128 : 64, 1, 0x7fffffff)) != FA_OK)
-    return s;
+  // D <= 128: two Q tiles per CTA, 128-key tiles; D = 256: one Q tile, 64-key tiles
+  const bool wide = c.D == 256;
+  if ((s = fill_params(c, p, wide ? 1 : 2, wide ? 64 : 128, 1, 0x7fffffff)) != FA_OK) return s;
   if (p.num_units == 0) return FA_OK;
   const bool half = c.dt == FA_FP16;
+  if (c.D == 64) return half ? launch_fwd<Fwd64H>(p, dev, st) : launch_fwd<Fwd64B>(p, dev, st);
   if (c.D == 128) return half ? launch_fwd<Fwd128H>(p, dev, st) : launch_fwd<Fwd128B>(p, dev, st);
   return half ? launch_fwd<Fwd256H>(p, dev, st) : launch_fwd<Fwd256B>(p, dev, st);
 }
@@ -298,7 +304,7 @@ fa_status launch_combine(const float *o_part, const float *lse_part, int ns, lon
   return FA_OK;
 }
 
-int splitkv_bn(int D) { return D == 128 ? 128 : 64; }
+int splitkv_bn(int D) { return D == 256 ? 64 : 128; }
 
 }  // namespace
 
@@ -397,11 +403,18 @@ fa_status fa_fwd_splitkv(const void *q, const void *k, const void *v, void *out,
   p.o_part = static_cast<float *>(workspace);
   p.lse_part = p.o_part + (size_t)ns * rows * D;
   const bool half = dt == FA_FP16;
-  if (D == 128)
+  if (D == 64)
+    s = half ? launch_fwd<Spl64H>(p, dev, st) : launch_fwd<Spl64B>(p, dev, st);
+  else if (D == 128)
     s = half ? launch_fwd<Spl128H>(p, dev, st) : launch_fwd<Spl128B>(p, dev, st);
   else
     s = half ? launch_fwd<Spl256H>(p, dev, st) : launch_fwd<Spl256B>(p, dev, st);
   if (s != FA_OK) return s;
+  if (D == 64)
+    return half ? launch_combine<64, true>(p.o_part, p.lse_part, ns, rows, out, lse, Hq, Sq,
+                                           B * Sq, 1, st)
+                : launch_combine<64, false>(p.o_part, p.lse_part, ns, rows, out, lse, Hq, Sq,
+                                            B * Sq, 1, st);
   if (D == 128)
     return half ? launch_combine<128, true>(p.o_part, p.lse_part, ns, rows, out, lse, Hq, Sq,
                                             B * Sq, 1, st)

@@ -1214,7 +1214,7 @@ __global__ void __launch_bounds__(256) fa_combine_kernel(const float *__restrict
     constexpr int U = 8;
     for (int s0 = 0; s0 < ns; s0 += U) {
       float w[U];
-      float4 x[U][E / 4];
+      float x[U][E];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int s = s0 + u;
@@ -1222,34 +1222,48 @@ __global__ void __launch_bounds__(256) fa_combine_kernel(const float *__restrict
         if (s < ns) {
           const float ls = __ldg(lse_part + (long long)s * rows + r);
           w[u] = ls == -INFINITY ? 0.f : ex2_approx((ls - Lse) * L2E);
-          const float4 *src =
-              reinterpret_cast<const float4 *>(o_part + ((long long)s * rows + r) * D + lane * E);
+          const float *src = o_part + ((long long)s * rows + r) * D + lane * E;
+          if constexpr (E % 4 == 0) {
 #pragma unroll
-          for (int e = 0; e < E / 4; ++e) x[u][e] = __ldg(src + e);
+            for (int e = 0; e < E; e += 4) {
+              const float4 v = __ldg(reinterpret_cast<const float4 *>(src + e));
+              x[u][e] = v.x;
+              x[u][e + 1] = v.y;
+              x[u][e + 2] = v.z;
+              x[u][e + 3] = v.w;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < E; e += 2) {
+              const float2 v = __ldg(reinterpret_cast<const float2 *>(src + e));
+              x[u][e] = v.x;
+              x[u][e + 1] = v.y;
+            }
+          }
         } else {
 #pragma unroll
-          for (int e = 0; e < E / 4; ++e) x[u][e] = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int e = 0; e < E; ++e) x[u][e] = 0.f;
         }
       }
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
+      for (int u = 0; u < U; ++u)
 #pragma unroll
-        for (int e = 0; e < E / 4; ++e) {
-          acc[4 * e] += w[u] * x[u][e].x;
-          acc[4 * e + 1] += w[u] * x[u][e].y;
-          acc[4 * e + 2] += w[u] * x[u][e].z;
-          acc[4 * e + 3] += w[u] * x[u][e].w;
-        }
-      }
+        for (int e = 0; e < E; ++e) acc[e] += w[u] * x[u][e];
     }
   }
   uint16_t *dst = reinterpret_cast<uint16_t *>(out) + r * D + lane * E;
+  if constexpr (E % 4 == 0) {
 #pragma unroll
-  for (int e = 0; e < E; e += 4) {
-    uint2 w;
-    w.x = pack2<HALF>(acc[e], acc[e + 1]);
-    w.y = pack2<HALF>(acc[e + 2], acc[e + 3]);
-    *reinterpret_cast<uint2 *>(dst + e) = w;
+    for (int e = 0; e < E; e += 4) {
+      uint2 w;
+      w.x = pack2<HALF>(acc[e], acc[e + 1]);
+      w.y = pack2<HALF>(acc[e + 2], acc[e + 3]);
+      *reinterpret_cast<uint2 *>(dst + e) = w;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < E; e += 2)
+      *reinterpret_cast<uint32_t *>(dst + e) = pack2<HALF>(acc[e], acc[e + 1]);
   }
   if (lane == 0 && lse != nullptr) {
     const long long tok = r / Hq;

@@ -19,6 +19,8 @@ Workloads (shapes from the pages' validation tables and API contracts):
   ("flashrt/fa4-cute-runtime", forward_static with seqused_k).
 * ``decode_splitkv``: B=8, Sq=1, Sk=131072, Hq=32, Hkv=8, D=128 split-KV
   decode with an LSE combine.
+* ``dense_d64``: dense non-causal MHA, B=4, S=4096, H=16, D=64 (a 64-wide
+  head dim, one of the small head dims the pages list as the next step).
 
 Seeds are 440410 + workload index (the seed style of the pages' benchmark).
 Values are drawn in float32 as N(0, 1) and rounded to the input dtype.
@@ -34,7 +36,7 @@ import torch
 SEED_BASE = 440410
 
 WORKLOADS = ["dense_257", "varlen_gqa_bias", "video_dit_20480",
-             "encoder_d256_seqused", "decode_splitkv"]
+             "encoder_d256_seqused", "decode_splitkv", "dense_d64"]
 
 _CHUNK = 1 << 24
 
@@ -197,6 +199,13 @@ def make(name: str, dtype=torch.bfloat16, device="cpu", decode_sk: int = 131072)
         v = _randn((B, Sk, Hkv, D), g, dtype)
         return Problem(name, "dense", q, k, v, softmax_scale=1 / math.sqrt(D),
                        max_seqlen_q=Sq, max_seqlen_k=Sk, splitkv=True)
+    if name == "dense_d64":
+        B, S, H, D = 4, 4096, 16, 64
+        q = _randn((B, S, H, D), g, dtype)
+        k = _randn((B, S, H, D), g, dtype)
+        v = _randn((B, S, H, D), g, dtype)
+        return Problem(name, "dense", q, k, v, softmax_scale=1 / math.sqrt(D),
+                       max_seqlen_q=S, max_seqlen_k=S)
     raise KeyError(name)
 
 

@@ -33,7 +33,7 @@
  *     synchronises the stream: a call only enqueues work on `stream`
  *     (a cudaStream_t; NULL means the legacy default stream) and returns.
  *   - Element type `dt` applies to q, k, v, out and rel_bias alike.
- *   - head_dim D must be 128 or 256; Hq must be a multiple of Hkv; query head
+ *   - head_dim D must be 64, 128 or 256; Hq must be a multiple of Hkv; query head
  *     h reads K/V head h / (Hq / Hkv).
  *   - q, k, v, out and rel_bias must be 16-byte aligned and contiguous in the
  *     documented layout.  cu_seqlens and seqused_k are device int32 arrays.

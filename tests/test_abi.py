@@ -55,7 +55,8 @@ def _fwd(lib, q=A, k=A, v=A, out=A, lse=A, B=1, Sq=16, Sk=16, Hq=4, Hkv=2, D=128
 
 
 def test_validation_statuses(lib):
-    assert _fwd(lib, D=64) == FA_ERR_UNSUPPORTED
+    assert _fwd(lib, D=96) == FA_ERR_UNSUPPORTED
+    assert _fwd(lib, D=32) == FA_ERR_UNSUPPORTED
     assert _fwd(lib, D=192) == FA_ERR_UNSUPPORTED
     assert _fwd(lib, Hq=6, Hkv=4) == FA_ERR_INVALID
     assert _fwd(lib, dt=7) == FA_ERR_INVALID
@@ -84,7 +85,7 @@ def test_varlen_validation(lib):
     r = lib.fa_fwd_varlen(A, A, A, A, A, None, None, None, 2, 8, 8, 16, 16, 4, 2,
                           128, 0, 0, 0.0, None, 0, None)
     assert r == FA_ERR_INVALID  # cu_seqlens missing
-    r = lib.fa_fwd_varlen(A, A, A, A, A, A, A, P, 2, 8, 8, 16, 16, 4, 2, 64, 0, 0,
+    r = lib.fa_fwd_varlen(A, A, A, A, A, A, A, P, 2, 8, 8, 16, 16, 4, 2, 96, 0, 0,
                           0.0, None, 0, None)
     assert r == FA_ERR_UNSUPPORTED
 

@@ -70,7 +70,7 @@ def test_dense_257(dtype):
 
 
 # ---------------------------------------------------------------------------
-# dense shapes: causal, Sq != Sk both ways, GQA groups, D = 128 / 256
+# dense shapes: causal, Sq != Sk both ways, GQA groups, D = 64 / 128 / 256
 # ---------------------------------------------------------------------------
 CASES = [
     # B, Sq, Sk, Hq, Hkv, D, causal
@@ -82,6 +82,8 @@ CASES = [
     (2, 200, 300, 8, 8, 256, False),
     (1, 300, 300, 8, 1, 256, True),    # D=256, group of 8 packed
     (1, 70, 600, 4, 4, 256, True),
+    (2, 300, 300, 4, 4, 64, True),     # D=64
+    (1, 129, 390, 8, 2, 64, False),    # D=64, group of 4 packed
 ]
 
 
@@ -94,7 +96,7 @@ def test_dense_shapes(case):
     compare(out, lse, ro, rl, what=str(case))
 
 
-@pytest.mark.parametrize("D", [128, 256])
+@pytest.mark.parametrize("D", [64, 128, 256])
 def test_fp16_causal_gqa(D):
     p = fa_inputs.random_dense(7, 2, 260, 270, 8, 2, D, dtype=torch.float16, causal=True)
     out, lse = run_dense(p)
@@ -105,7 +107,7 @@ def test_fp16_causal_gqa(D):
 # ---------------------------------------------------------------------------
 # varlen with empty / one-token / multi-tile sequences, causal, GQA, bias
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("D", [128, 256])
+@pytest.mark.parametrize("D", [64, 128, 256])
 @pytest.mark.parametrize("causal", [False, True])
 def test_varlen_bias(D, causal):
     q_lens = [0, 1, 130, 257, 513, 64]
@@ -191,12 +193,23 @@ def test_video_dit_20480_sampled():
     gl = np.array([float(l[b, h, i]) for b, h, i in rows])
     compare(go, gl, ro, rl, what="video_dit sampled")
 
+def test_dense_d64_sampled():
+    p = fa_inputs.make("dense_d64")
+    out, lse = run_dense(p)
+    rows = _sample_rows(np.random.default_rng(2), 4, 16, [4096] * 4, 256)
+    ro, rl = oracle.attention_rows(p.q, p.k, p.v, rows, softmax_scale=p.softmax_scale)
+    o = out.float().cpu()
+    l = lse.cpu()
+    go = np.stack([o[b, i, h].numpy() for b, h, i in rows])
+    gl = np.array([float(l[b, h, i]) for b, h, i in rows])
+    compare(go, gl, ro, rl, what="dense_d64 sampled")
+
 
 # ---------------------------------------------------------------------------
 # split-KV
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("ns", [0, 1, 3, 7])
-@pytest.mark.parametrize("D", [128, 256])
+@pytest.mark.parametrize("D", [64, 128, 256])
 def test_splitkv_small(ns, D):
     p = fa_inputs.random_dense(21 + D, 3, 1, 1000, 8, 2, D)
     g = p.to(DEV)
@@ -312,7 +325,7 @@ def test_many_batches_beyond_grid_y_limit():
 
 
 def test_invalid_arguments_raise_and_write_nothing():
-    q = torch.randn(1, 16, 4, 64, device=DEV, dtype=torch.bfloat16)
+    q = torch.randn(1, 16, 4, 96, device=DEV, dtype=torch.bfloat16)
     with pytest.raises(fa.FAError) as e:
         fa.fa_fwd(q, q, q)
     assert e.value.name == "FA_ERR_UNSUPPORTED"
