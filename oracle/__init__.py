@@ -14,6 +14,9 @@ rows); this module only marshals arrays into it.  It follows the pages:
   K/V length of a padded buffer.
 * "FlashAttention-4 backend for Blackwell #1235": combining key-range splits
   through the LSE.
+* "mgoin/tml-fa4" lists mask/score modifiers without defining them; the
+  sliding window and soft-cap here are the plainest readings (see
+  ``fa_oracle.c``).
 
 Layouts: dense q [B, Sq, Hq, D], k/v [B, Sk, Hkv, D], out like q, lse
 [B, Hq, Sq]; varlen q [total_q, Hq, D], k/v [total_k, Hkv, D], lse
@@ -57,11 +60,13 @@ def _load():
         i32 = ctypes.c_int
         lib.fa_oracle_forward.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32,
                                           i32, ctypes.c_double, P, i32, i32,
-                                          i32, P, P, i32]
+                                          i32, P, P, i32, i32, i32,
+                                          ctypes.c_double]
         lib.fa_oracle_forward.restype = i32
         lib.fa_oracle_rows.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32,
                                        i32, ctypes.c_double, P, i32, P, P, P,
-                                       ctypes.c_long, P, P, i32]
+                                       ctypes.c_long, P, P, i32, i32, i32,
+                                       ctypes.c_double]
         lib.fa_oracle_rows.restype = i32
         lib.fa_oracle_lse_combine.argtypes = [P, P, i32, ctypes.c_long, i32,
                                               P, P]
@@ -134,11 +139,15 @@ def _as_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, rel_bias):
 
 def attention(q, k, v, *, cu_seqlens_q=None, cu_seqlens_k=None,
               seqused_k=None, causal: bool = False, softmax_scale=None,
-              rel_bias=None, kv_range=None, nthreads: int = 0):
+              rel_bias=None, kv_range=None, window=(-1, -1), softcap: float = 0.0,
+              nthreads: int = 0):
     """Exact attention of every row; returns (out, lse) as float64 arrays.
 
     ``kv_range=(lo, hi)`` restricts every sequence to its keys [lo, hi) and
     returns that split's partial (O normalised over the range, and its LSE).
+    ``window=(left, right)`` masks keys more than ``left`` before / ``right``
+    after the row's diagonal (negative: no bound); ``softcap > 0`` maps each
+    scaled score s to softcap * tanh(s / softcap) before the bias.
     """
     q, k, v = _f32(q), _f32(k), _f32(v)
     rel_bias = _f32(rel_bias)
@@ -154,7 +163,8 @@ def attention(q, k, v, *, cu_seqlens_q=None, cu_seqlens_k=None,
     rc = _load().fa_oracle_forward(
         _ptr(q), _ptr(k), _ptr(v), _ptr(cu_q), _ptr(cu_k), _ptr(su), B, Hq,
         Hkv, D, int(bool(causal)), _default_scale(D, softmax_scale),
-        _ptr(rel_bias), R, int(lo), int(hi), _ptr(out), _ptr(lse), nthreads)
+        _ptr(rel_bias), R, int(lo), int(hi), _ptr(out), _ptr(lse), nthreads,
+        int(window[0]), int(window[1]), float(softcap))
     if rc:
         raise ValueError(f"oracle rejected the problem (code {rc})")
     if dense:
@@ -166,7 +176,8 @@ def attention(q, k, v, *, cu_seqlens_q=None, cu_seqlens_k=None,
 
 def attention_rows(q, k, v, rows, *, cu_seqlens_q=None, cu_seqlens_k=None,
                    seqused_k=None, causal: bool = False, softmax_scale=None,
-                   rel_bias=None, nthreads: int = 0):
+                   rel_bias=None, window=(-1, -1), softcap: float = 0.0,
+                   nthreads: int = 0):
     """Exact attention of chosen rows only.
 
     ``rows`` is an int array [n, 3] of (b, h, i): batch, query head and query
@@ -191,7 +202,7 @@ def attention_rows(q, k, v, rows, *, cu_seqlens_q=None, cu_seqlens_k=None,
         _ptr(q), _ptr(k), _ptr(v), _ptr(cu_q), _ptr(cu_k), _ptr(su), B, Hq,
         Hkv, D, int(bool(causal)), _default_scale(D, softmax_scale),
         _ptr(rel_bias), R, _ptr(rb), _ptr(rh), _ptr(ri), n, _ptr(out),
-        _ptr(lse), nthreads)
+        _ptr(lse), nthreads, int(window[0]), int(window[1]), float(softcap))
     if rc:
         raise ValueError(f"oracle rejected the rows (code {rc})")
     return out, lse

@@ -31,6 +31,16 @@
  *   - the LSE is the natural logarithm;
  *   - a row with no admissible key gets O = 0 and LSE = -inf.
  *
+ * Score and mask modifiers ("mgoin/tml-fa4" lists "mask/score modifiers"
+ * among the forward paths without defining them; these are the plainest
+ * readings, listed with the design notes):
+ *   - sliding window: with d the distance above, a key is masked when
+ *     d > window_left (too far left of the row's diagonal, window_left >= 0)
+ *     or -d > window_right (too far right, window_right >= 0); a negative
+ *     bound is no bound, and causal mode is window_right = 0;
+ *   - soft-capping: with cap > 0 the scaled score s becomes cap * tanh(s / cap)
+ *     before the bias is added.
+ *
  * Inputs arrive as float arrays holding the exact bf16/fp16 input values
  * (both formats embed exactly in binary32); every product, sum, exponential
  * and logarithm below is done in double.
@@ -55,6 +65,8 @@ typedef struct {
   const float *rel_bias;        /* [total_q,Hq,R] or NULL */
   int B, Hq, Hkv, D, R, causal;
   double scale;
+  int window_left, window_right; /* < 0: no bound */
+  double softcap;                /* > 0: cap * tanh(s / cap); 0: off */
 } fa_problem;
 
 /* One attention row: batch b, query head h, query position i (0-based within
@@ -81,7 +93,8 @@ static long attend_row(const fa_problem *p, int b, int h, int i, int kv_lo,
   long n_ok = 0;
   for (int j = lo; j < hi; ++j) {
     long d = (long)i + delta - (long)j;
-    if (p->causal && d < 0) {
+    if ((p->causal && d < 0) || (p->window_left >= 0 && d > p->window_left) ||
+        (p->window_right >= 0 && -d > p->window_right)) {
       s_scratch[j - lo] = -INFINITY;
       continue;
     }
@@ -89,6 +102,7 @@ static long attend_row(const fa_problem *p, int b, int h, int i, int kv_lo,
     double acc = 0.0;
     for (int t = 0; t < D; ++t) acc += (double)qv[t] * (double)kv[t];
     double s = p->scale * acc;
+    if (p->softcap > 0.0) s = p->softcap * tanh(s / p->softcap);
     if (p->rel_bias && d >= 0 && d < p->R)
       s += (double)p->rel_bias[(qrow * p->Hq + h) * (long)p->R + d];
     s_scratch[j - lo] = s;
@@ -128,6 +142,7 @@ static int check_problem(const fa_problem *p) {
   if (p->B < 0 || p->Hq <= 0 || p->Hkv <= 0 || p->D <= 0) return 1;
   if (p->Hq % p->Hkv) return 2;
   if (p->rel_bias && p->R <= 0) return 3;
+  if (!(p->softcap >= 0.0)) return 8;
   for (int b = 0; b < p->B; ++b) {
     if (p->cu_q[b + 1] < p->cu_q[b] || p->cu_k[b + 1] < p->cu_k[b]) return 4;
     if (p->seqused_k && (p->seqused_k[b] < 0 ||
@@ -147,9 +162,10 @@ int fa_oracle_forward(const float *q, const float *k, const float *v,
                       const int *cu_q, const int *cu_k, const int *seqused_k,
                       int B, int Hq, int Hkv, int D, int causal, double scale,
                       const float *rel_bias, int R, int kv_lo, int kv_hi,
-                      double *out, double *lse, int nthreads) {
+                      double *out, double *lse, int nthreads, int window_left,
+                      int window_right, double softcap) {
   fa_problem p = {q, k, v, cu_q, cu_k, seqused_k, rel_bias, B, Hq, Hkv, D, R,
-                  causal, scale};
+                  causal, scale, window_left, window_right, softcap};
   int rc = check_problem(&p);
   if (rc) return rc;
   const long total_q = B > 0 ? cu_q[B] : 0;
@@ -195,9 +211,10 @@ int fa_oracle_rows(const float *q, const float *k, const float *v,
                    int B, int Hq, int Hkv, int D, int causal, double scale,
                    const float *rel_bias, int R, const int *row_b,
                    const int *row_h, const int *row_i, long n_rows,
-                   double *out, double *lse, int nthreads) {
+                   double *out, double *lse, int nthreads, int window_left,
+                   int window_right, double softcap) {
   fa_problem p = {q, k, v, cu_q, cu_k, seqused_k, rel_bias, B, Hq, Hkv, D, R,
-                  causal, scale};
+                  causal, scale, window_left, window_right, softcap};
   int rc = check_problem(&p);
   if (rc) return rc;
   for (long r = 0; r < n_rows; ++r) {

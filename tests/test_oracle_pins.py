@@ -368,3 +368,88 @@ def test_workload_shapes_match_their_descriptions():
     # 1e4 rounded to bf16
     pad = float(torch.tensor(1e4).to(torch.bfloat16))
     assert float(p.k[0, 968:].float().min()) == pad and float(p.v[1, 968:].float().max()) == pad
+
+
+# --------------------------------------------------------------------------
+# score and mask modifiers (readings of the pages' "mask/score modifiers"):
+# sliding window by distance d = i + (k_len - q_len) - j, soft-cap before bias
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("q_len,k_len,left,right,causal", [
+    (6, 6, 2, 1, False),    # window both sides
+    (5, 9, 3, -1, False),   # left bound only, k longer (delta = 4)
+    (7, 4, -1, 2, False),   # right bound only, k shorter (delta = -3)
+    (6, 8, 1, 5, True),     # causal caps the right side at 0
+    (8, 8, 0, 0, False),    # the diagonal key alone
+])
+def test_window_weights_are_uniform_over_the_admissible_band(q_len, k_len, left, right, causal):
+    # q = 0: every admissible key has score 0, so with one-hot values each
+    # output row is 1/count on the admissible keys and LSE = ln(count)
+    D = max(k_len, 1)
+    q = np.zeros((q_len, 1, D), dtype=np.float32)
+    k = np.random.default_rng(5).standard_normal((k_len, 1, D)).astype(np.float32)
+    v = _one_hot_v(k_len, D)
+    cu_q = np.array([0, q_len], dtype=np.int32)
+    cu_k = np.array([0, k_len], dtype=np.int32)
+    out, lse = oracle.attention(q, k, v, cu_seqlens_q=cu_q, cu_seqlens_k=cu_k,
+                                causal=causal, window=(left, right))
+    delta = k_len - q_len
+    for i in range(q_len):
+        ok = []
+        for j in range(k_len):
+            d = i + delta - j
+            if causal and d < 0:
+                continue
+            if left >= 0 and d > left:
+                continue
+            if right >= 0 and -d > right:
+                continue
+            ok.append(j)
+        want = np.zeros(D)
+        for j in ok:
+            want[j] = 1.0 / len(ok)
+        np.testing.assert_allclose(out[i, 0], want, atol=1e-15)
+        if ok:
+            assert lse[0, i] == pytest.approx(math.log(len(ok)), abs=1e-14)
+        else:
+            assert lse[0, i] == -math.inf
+
+
+def test_softcap_single_key_closed_form_and_order_with_bias():
+    # D = 1, q = 2, k = 3, scale 1: raw score 6; one key, so LSE is the score
+    q = np.full((1, 1, 1), 2.0, dtype=np.float32)
+    k = np.full((1, 1, 1), 3.0, dtype=np.float32)
+    v = np.full((1, 1, 1), 0.75, dtype=np.float32)
+    cu = np.array([0, 1], dtype=np.int32)
+    for cap in (4.0, 10.0, 0.5):
+        out, lse = oracle.attention(q, k, v, cu_seqlens_q=cu, cu_seqlens_k=cu,
+                                    softmax_scale=1.0, softcap=cap)
+        assert out[0, 0, 0] == pytest.approx(0.75, abs=1e-15)
+        assert lse[0, 0] == pytest.approx(cap * math.tanh(6.0 / cap), abs=1e-13)
+    # the bias (distance 0) is added after the cap, unscaled
+    rb = np.full((1, 1, 128), 0.0, dtype=np.float32)
+    rb[0, 0, 0] = -1.25
+    out, lse = oracle.attention(q, k, v, cu_seqlens_q=cu, cu_seqlens_k=cu,
+                                softmax_scale=1.0, softcap=4.0, rel_bias=rb)
+    assert lse[0, 0] == pytest.approx(4.0 * math.tanh(1.5) - 1.25, abs=1e-13)
+
+
+def test_softcap_saturates_and_vanishes_in_the_limit():
+    # raw scores +1e6 and -1e6 cap to +c and -c: weights 1/(1 + e^{-2c})
+    q = np.full((1, 1, 2), 1.0, dtype=np.float32)
+    k = np.array([[[1e6, 0.0]], [[-1e6, 0.0]]], dtype=np.float32)
+    v = _one_hot_v(2, 2)
+    cu_q = np.array([0, 1], dtype=np.int32)
+    cu_k = np.array([0, 2], dtype=np.int32)
+    c = 1.5
+    out, lse = oracle.attention(q, k, v, cu_seqlens_q=cu_q, cu_seqlens_k=cu_k,
+                                softmax_scale=1.0, softcap=c)
+    w1 = 1.0 / (1.0 + math.exp(-2 * c))
+    np.testing.assert_allclose(out[0, 0], [w1, 1.0 - w1], atol=1e-15)
+    assert lse[0, 0] == pytest.approx(c + math.log1p(math.exp(-2 * c)), abs=1e-13)
+    # a cap far above the scores leaves them as they are
+    k2 = np.array([[[0.5, 0.0]], [[-0.25, 0.0]]], dtype=np.float32)
+    out, lse = oracle.attention(q, k2, v, cu_seqlens_q=cu_q, cu_seqlens_k=cu_k,
+                                softmax_scale=1.0, softcap=1e9)
+    z = math.exp(0.5) + math.exp(-0.25)
+    np.testing.assert_allclose(out[0, 0], [math.exp(0.5) / z, math.exp(-0.25) / z], atol=1e-12)
+    assert lse[0, 0] == pytest.approx(math.log(z), abs=1e-12)
