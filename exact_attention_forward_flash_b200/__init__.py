@@ -45,6 +45,17 @@ class FAError(RuntimeError):
         self.name = name
 
 
+class FaMods(ctypes.Structure):
+    """Mirror of fa_mods (include/fa_b200.h)."""
+    _fields_ = [("window_left", ctypes.c_int), ("window_right", ctypes.c_int),
+                ("softcap", ctypes.c_float)]
+
+
+def _mods(window, softcap):
+    wl, wr = (-1, -1) if window is None else (int(window[0]), int(window[1]))
+    return FaMods(wl, wr, float(softcap or 0.0))
+
+
 def load_library(path: Optional[str] = None):
     """Load the shared library (raises if it is absent)."""
     global _lib
@@ -74,6 +85,13 @@ def load_library(path: Optional[str] = None):
     lib.fa_fwd_splitkv_static.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32,
                                           i32, i32, i32, f32, P, P, i32, i32, P]
     lib.fa_fwd_splitkv_static.restype = i32
+    M = ctypes.POINTER(FaMods)
+    lib.fa_fwd_ex.argtypes = lib.fa_fwd.argtypes[:-1] + [M, P]
+    lib.fa_fwd_ex.restype = i32
+    lib.fa_fwd_varlen_ex.argtypes = lib.fa_fwd_varlen.argtypes[:-1] + [M, P]
+    lib.fa_fwd_varlen_ex.restype = i32
+    lib.fa_fwd_splitkv_ex.argtypes = lib.fa_fwd_splitkv.argtypes[:-1] + [M, P]
+    lib.fa_fwd_splitkv_ex.restype = i32
     lib.fa_check_device_error.argtypes = [ctypes.POINTER(i32), i32]
     lib.fa_check_device_error.restype = i32
     lib.fa_status_string.argtypes = [i32]
@@ -138,8 +156,11 @@ def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
            rel_bias: Optional[torch.Tensor] = None,
            out: Optional[torch.Tensor] = None,
            lse: Optional[torch.Tensor] = None,
+           window: Optional[Tuple[int, int]] = None, softcap: float = 0.0,
            stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Dense forward: q [B,Sq,Hq,D], k/v [B,Sk,Hkv,D] -> (out, lse [B,Hq,Sq])."""
+    """Dense forward: q [B,Sq,Hq,D], k/v [B,Sk,Hkv,D] -> (out, lse [B,Hq,Sq]).
+
+    ``window=(left, right)`` and ``softcap`` are the fa_mods modifiers."""
     lib = load_library()
     B, Sq, Hq, D = q.shape
     _, Sk, Hkv, _ = k.shape
@@ -153,10 +174,11 @@ def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
     _same_dtype(q, k, v, out, rel_bias)
     _int32(seqused_k, "seqused_k")
     R = 0 if rel_bias is None else int(rel_bias.shape[-1])
-    _check(lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq,
-                      Sk, Hq, Hkv, D, _dtype(q), int(bool(causal)),
-                      float(softmax_scale or 0.0), _ptr(seqused_k),
-                      _ptr(rel_bias), R, _stream(stream)))
+    m = _mods(window, softcap)
+    _check(lib.fa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq,
+                         Sk, Hq, Hkv, D, _dtype(q), int(bool(causal)),
+                         float(softmax_scale or 0.0), _ptr(seqused_k),
+                         _ptr(rel_bias), R, ctypes.byref(m), _stream(stream)))
     return out, lse
 
 
@@ -168,6 +190,7 @@ def fa_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                   rel_bias: Optional[torch.Tensor] = None,
                   out: Optional[torch.Tensor] = None,
                   lse: Optional[torch.Tensor] = None,
+                  window: Optional[Tuple[int, int]] = None, softcap: float = 0.0,
                   stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Varlen forward: q [total_q,Hq,D], k/v [total_k,Hkv,D] ->
     (out [total_q,Hq,D], lse [Hq,total_q])."""
@@ -185,12 +208,13 @@ def fa_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                  (seqused_k, "seqused_k")):
         _int32(t, n)
     R = 0 if rel_bias is None else int(rel_bias.shape[-1])
-    _check(lib.fa_fwd_varlen(
+    m = _mods(window, softcap)
+    _check(lib.fa_fwd_varlen_ex(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens_q),
         _ptr(cu_seqlens_k), _ptr(seqused_k), B, int(max_seqlen_q),
         int(max_seqlen_k), total_q, total_k, Hq, Hkv, D, _dtype(q),
         int(bool(causal)), float(softmax_scale or 0.0), _ptr(rel_bias), R,
-        _stream(stream)))
+        ctypes.byref(m), _stream(stream)))
     return out, lse
 
 
@@ -210,6 +234,7 @@ def fa_fwd_splitkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
                    out: Optional[torch.Tensor] = None,
                    lse: Optional[torch.Tensor] = None,
                    workspace: Optional[torch.Tensor] = None,
+                   window: Optional[Tuple[int, int]] = None, softcap: float = 0.0,
                    stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Split-KV dense forward (decode); returns (out, lse [B,Hq,Sq])."""
     lib = load_library()
@@ -230,11 +255,13 @@ def fa_fwd_splitkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
     _same_dtype(q, k, v, out, rel_bias)
     _int32(seqused_k, "seqused_k")
     R = 0 if rel_bias is None else int(rel_bias.shape[-1])
-    _check(lib.fa_fwd_splitkv(
+    m = _mods(window, softcap)
+    _check(lib.fa_fwd_splitkv_ex(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq, Sk, Hq, Hkv,
         D, _dtype(q), int(bool(causal)), float(softmax_scale or 0.0),
         _ptr(seqused_k), _ptr(rel_bias), R, int(ns), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _stream(stream)))
+        workspace.numel() * workspace.element_size(), ctypes.byref(m),
+        _stream(stream)))
     return out, lse
 
 

@@ -128,18 +128,13 @@ int num_sms(int dev) {
 }
 
 // kernel variants
-using Fwd64B = FwdCfg<64, 128, 2, 1, 3, 0, false, false>;
-using Fwd64H = FwdCfg<64, 128, 2, 1, 3, 0, true, false>;
-using Fwd128B = FwdCfg<128, 128, 2, 1, 3, 0, false, false>;
-using Fwd128H = FwdCfg<128, 128, 2, 1, 3, 0, true, false>;
-using Fwd256B = FwdCfg<256, 64, 1, 2, 3, 2, false, false>;
-using Fwd256H = FwdCfg<256, 64, 1, 2, 3, 2, true, false>;
-using Spl64B = FwdCfg<64, 128, 1, 2, 3, 3, false, true>;
-using Spl64H = FwdCfg<64, 128, 1, 2, 3, 3, true, true>;
-using Spl128B = FwdCfg<128, 128, 1, 2, 3, 3, false, true>;
-using Spl128H = FwdCfg<128, 128, 1, 2, 3, 3, true, true>;
-using Spl256B = FwdCfg<256, 64, 1, 2, 2, 2, false, true>;
-using Spl256H = FwdCfg<256, 64, 1, 2, 2, 2, true, true>;
+// kernel configurations by (16-bit format: bf16 / fp16, modifiers off / on)
+template <bool H, bool M> using Fwd64 = FwdCfg<64, 128, 2, 1, 3, 0, H, false, M>;
+template <bool H, bool M> using Fwd128 = FwdCfg<128, 128, 2, 1, 3, 0, H, false, M>;
+template <bool H, bool M> using Fwd256 = FwdCfg<256, 64, 1, 2, 3, 2, H, false, M>;
+template <bool H, bool M> using Spl64 = FwdCfg<64, 128, 1, 2, 3, 3, H, true, M>;
+template <bool H, bool M> using Spl128 = FwdCfg<128, 128, 1, 2, 3, 3, H, true, M>;
+template <bool H, bool M> using Spl256 = FwdCfg<256, 64, 1, 2, 2, 2, H, true, M>;
 
 template <class C>
 fa_status launch_fwd(FwdParams &p, int dev, cudaStream_t st) {
@@ -161,6 +156,17 @@ fa_status launch_fwd(FwdParams &p, int dev, cudaStream_t st) {
   return FA_OK;
 }
 
+// one of the four variants of a configuration
+template <template <bool, bool> class Cfg>
+fa_status launch_variant(FwdParams &p, int dev, cudaStream_t st, bool half, bool mods) {
+  if (half) return mods ? launch_fwd<Cfg<true, true>>(p, dev, st) : launch_fwd<Cfg<true, false>>(p, dev, st);
+  return mods ? launch_fwd<Cfg<false, true>>(p, dev, st) : launch_fwd<Cfg<false, false>>(p, dev, st);
+}
+
+// the modifier kernels serve a left window bound or a soft-cap (the plain
+// ones serve causal masking and any right window bound)
+bool uses_mods(const FwdParams &p) { return p.wl >= 0 || p.cap_a > 0.f; }
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 constexpr unsigned long long kTimeoutNs = 4000000000ull;  // 4 s per wait
@@ -176,7 +182,17 @@ struct Common {
   int causal;
   float scale;
   bool varlen;
+  // modifiers (fa_mods): window bounds (< 0: none), soft-cap (0: off)
+  int window_left = -1, window_right = -1;
+  float softcap = 0.f;
 };
+
+void apply_mods(Common &c, const fa_mods *m) {
+  if (m == nullptr) return;
+  c.window_left = m->window_left;
+  c.window_right = m->window_right;
+  c.softcap = m->softcap;
+}
 
 fa_status validate(const Common &c) {
   if (c.dt != FA_BF16 && c.dt != FA_FP16) return fail(FA_ERR_INVALID, "dtype must be bf16 or fp16");
@@ -197,6 +213,8 @@ fa_status validate(const Common &c) {
       return fail(FA_ERR_UNSUPPORTED, "rel_bias larger than 64 GiB");
   }
   if (!std::isfinite(c.scale)) return fail(FA_ERR_INVALID, "softmax_scale must be finite");
+  if (!std::isfinite(c.softcap) || c.softcap < 0.f)
+    return fail(FA_ERR_INVALID, "softcap must be finite and >= 0");
   const long long tq = c.varlen ? c.total_q : (long long)c.B * c.Sq;
   const long long tk = c.varlen ? c.total_k : (long long)c.B * c.Sk;
   if (tq > 0x7fffffffLL || tk > 0x7fffffffLL || tq * c.Hq > (1LL << 40))
@@ -268,6 +286,12 @@ fa_status fill_params(const Common &c, FwdParams &p, int nq, int bn, int num_spl
   p.scale_log2 = scale * 1.4426950408889634f;
   p.inv_scale = 1.0f / scale;
   p.thr_raw = 8.0f / p.scale_log2;
+  p.wl = c.window_left < 0 ? -1 : c.window_left;
+  p.wr = c.causal ? 0 : (c.window_right < 0 ? -1 : c.window_right);
+  if (c.softcap > 0.f) {
+    p.cap_a = c.softcap / scale;  // raw-score units
+    p.cap_b = scale / c.softcap;
+  }
   p.timeout_ns = kTimeoutNs;
   return FA_OK;
 }
@@ -285,9 +309,10 @@ fa_status run_fwd(const Common &c, cudaStream_t st) {
   if ((s = fill_params(c, p, wide ? 1 : 2, wide ? 64 : 128, 1, 0x7fffffff)) != FA_OK) return s;
   if (p.num_units == 0) return FA_OK;
   const bool half = c.dt == FA_FP16;
-  if (c.D == 64) return half ? launch_fwd<Fwd64H>(p, dev, st) : launch_fwd<Fwd64B>(p, dev, st);
-  if (c.D == 128) return half ? launch_fwd<Fwd128H>(p, dev, st) : launch_fwd<Fwd128B>(p, dev, st);
-  return half ? launch_fwd<Fwd256H>(p, dev, st) : launch_fwd<Fwd256B>(p, dev, st);
+  const bool mods = uses_mods(p);
+  if (c.D == 64) return launch_variant<Fwd64>(p, dev, st, half, mods);
+  if (c.D == 128) return launch_variant<Fwd128>(p, dev, st, half, mods);
+  return launch_variant<Fwd256>(p, dev, st, half, mods);
 }
 
 template <int D, bool HALF>
@@ -326,13 +351,36 @@ const char *fa_last_error_message(void) { return g_msg; }
 
 const char *fa_version(void) { return "fa_b200 0.1 (sm_100a)"; }
 
+fa_status fa_fwd_ex(const void *q, const void *k, const void *v, void *out, float *lse, int B,
+                    int Sq, int Sk, int Hq, int Hkv, int D, fa_dtype dt, int causal,
+                    float softmax_scale, const int *seqused_k, const void *rel_bias,
+                    int rel_extent, const fa_mods *mods, void *stream) {
+  g_msg[0] = 0;
+  Common c{q, k, v, out, lse, nullptr, nullptr, seqused_k, rel_bias, rel_extent, B, Sq, Sk,
+           Hq, Hkv, D, 0, 0, 0, dt, causal, softmax_scale, false};
+  apply_mods(c, mods);
+  return run_fwd(c, static_cast<cudaStream_t>(stream));
+}
+
 fa_status fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse, int B,
                  int Sq, int Sk, int Hq, int Hkv, int D, fa_dtype dt, int causal,
                  float softmax_scale, const int *seqused_k, const void *rel_bias, int rel_extent,
                  void *stream) {
+  return fa_fwd_ex(q, k, v, out, lse, B, Sq, Sk, Hq, Hkv, D, dt, causal, softmax_scale,
+                   seqused_k, rel_bias, rel_extent, nullptr, stream);
+}
+
+fa_status fa_fwd_varlen_ex(const void *q, const void *k, const void *v, void *out, float *lse,
+                           const int *cu_seqlens_q, const int *cu_seqlens_k,
+                           const int *seqused_k, int B, int max_seqlen_q, int max_seqlen_k,
+                           int total_q, int total_k, int Hq, int Hkv, int D, fa_dtype dt,
+                           int causal, float softmax_scale, const void *rel_bias,
+                           int rel_extent, const fa_mods *mods, void *stream) {
   g_msg[0] = 0;
-  Common c{q, k, v, out, lse, nullptr, nullptr, seqused_k, rel_bias, rel_extent, B, Sq, Sk,
-           Hq, Hkv, D, 0, 0, 0, dt, causal, softmax_scale, false};
+  (void)max_seqlen_k;
+  Common c{q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, seqused_k, rel_bias, rel_extent, B,
+           0, 0, Hq, Hkv, D, total_q, total_k, max_seqlen_q, dt, causal, softmax_scale, true};
+  apply_mods(c, mods);
   return run_fwd(c, static_cast<cudaStream_t>(stream));
 }
 
@@ -341,11 +389,9 @@ fa_status fa_fwd_varlen(const void *q, const void *k, const void *v, void *out, 
                         int B, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
                         int Hq, int Hkv, int D, fa_dtype dt, int causal, float softmax_scale,
                         const void *rel_bias, int rel_extent, void *stream) {
-  g_msg[0] = 0;
-  (void)max_seqlen_k;
-  Common c{q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, seqused_k, rel_bias, rel_extent, B,
-           0, 0, Hq, Hkv, D, total_q, total_k, max_seqlen_q, dt, causal, softmax_scale, true};
-  return run_fwd(c, static_cast<cudaStream_t>(stream));
+  return fa_fwd_varlen_ex(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, seqused_k, B,
+                          max_seqlen_q, max_seqlen_k, total_q, total_k, Hq, Hkv, D, dt, causal,
+                          softmax_scale, rel_bias, rel_extent, nullptr, stream);
 }
 
 size_t fa_splitkv_workspace_bytes(int B, int Sq, int Hq, int D, int num_splits) {
@@ -376,9 +422,21 @@ fa_status fa_fwd_splitkv(const void *q, const void *k, const void *v, void *out,
                          float softmax_scale, const int *seqused_k, const void *rel_bias,
                          int rel_extent, int num_splits, void *workspace, size_t workspace_bytes,
                          void *stream) {
+  return fa_fwd_splitkv_ex(q, k, v, out, lse, B, Sq, Sk, Hq, Hkv, D, dt, causal, softmax_scale,
+                           seqused_k, rel_bias, rel_extent, num_splits, workspace,
+                           workspace_bytes, nullptr, stream);
+}
+
+fa_status fa_fwd_splitkv_ex(const void *q, const void *k, const void *v, void *out, float *lse,
+                            int B, int Sq, int Sk, int Hq, int Hkv, int D, fa_dtype dt,
+                            int causal, float softmax_scale, const int *seqused_k,
+                            const void *rel_bias, int rel_extent, int num_splits,
+                            void *workspace, size_t workspace_bytes, const fa_mods *mods,
+                            void *stream) {
   g_msg[0] = 0;
   Common c{q, k, v, out, lse, nullptr, nullptr, seqused_k, rel_bias, rel_extent, B, Sq, Sk,
            Hq, Hkv, D, 0, 0, 0, dt, causal, softmax_scale, false};
+  apply_mods(c, mods);
   fa_status s = validate(c);
   if (s != FA_OK) return s;
   if (num_splits < 0) return fail(FA_ERR_INVALID, "num_splits must be >= 0");
@@ -404,11 +462,11 @@ fa_status fa_fwd_splitkv(const void *q, const void *k, const void *v, void *out,
   p.lse_part = p.o_part + (size_t)ns * rows * D;
   const bool half = dt == FA_FP16;
   if (D == 64)
-    s = half ? launch_fwd<Spl64H>(p, dev, st) : launch_fwd<Spl64B>(p, dev, st);
+    s = launch_variant<Spl64>(p, dev, st, half, uses_mods(p));
   else if (D == 128)
-    s = half ? launch_fwd<Spl128H>(p, dev, st) : launch_fwd<Spl128B>(p, dev, st);
+    s = launch_variant<Spl128>(p, dev, st, half, uses_mods(p));
   else
-    s = half ? launch_fwd<Spl256H>(p, dev, st) : launch_fwd<Spl256B>(p, dev, st);
+    s = launch_variant<Spl256>(p, dev, st, half, uses_mods(p));
   if (s != FA_OK) return s;
   if (D == 64)
     return half ? launch_combine<64, true>(p.o_part, p.lse_part, ns, rows, out, lse, Hq, Sq,

@@ -90,6 +90,19 @@ __device__ __forceinline__ float exp_pack(const float (&s)[M], float sl2, float 
   return (a + b) + (c + d);
 }
 
+// Soft-cap of N scores in raw-score units: x -> a * tanh(b * x), with tanh
+// from its definition, tanh(y) = sign(y) * (1 - 2 / (1 + e^(2|y|))), and
+// e^(2|y|) = 2^(2 log2(e) |y|) kept below overflow (tanh is 1 to fp32 there).
+template <int N>
+__device__ __forceinline__ void softcap_all(float (&x)[N], float a, float b) {
+#pragma unroll
+  for (int e = 0; e < N; ++e) {
+    const float y = b * x[e];
+    const float t = ex2_approx(fminf(2.8853900817779268f * fabsf(y), 126.f));
+    x[e] = copysignf(a * (1.f - __fdividef(2.f, 1.f + t)), y);
+  }
+}
+
 // Row max of the N columns [OFF, OFF + N) over four independent chains of
 // three-input maxima.
 template <int OFF, int N, int M>
@@ -122,6 +135,11 @@ struct FwdParams {
   int num_splits;
   int split_keys;    // keys per split (multiple of BN); >= any k_len when 1 split
   int causal;
+  // window by distance d = i + delta - j from the row's diagonal: a key is
+  // masked when d > wl (wl >= 0) or -d > wr (wr >= 0; causal makes wr 0)
+  int wl, wr;
+  // soft-cap in raw-score units: s -> cap_a * tanh(cap_b * s) when cap_a > 0
+  float cap_a, cap_b;
   int m_major;       // unit order: 1 = largest tile index first over all heads
   int compact;       // 1: causal units enumerated without empty ones (see Sched)
   int lse_dense;     // 1: lse [B, Hq, Sq]; 0: lse [Hq, total_q]
@@ -253,11 +271,17 @@ __device__ __forceinline__ bool decode_unit(const FwdParams &p, const Sched &sch
   for (int t = 0; t < NQ; ++t)
     if ((U.row0 + t * kBM) / p.P < U.q_len) U.active |= 1u << t;
   U.delta = U.k_len - U.q_len;
-  const long long lo = (long long)U.split * p.split_keys;
+  long long lo = (long long)U.split * p.split_keys;
   long long hi = min((long long)U.k_len, lo + p.split_keys);
-  if (p.causal) {
+  // keys no row of the unit admits are not visited: the window (causal is
+  // wr = 0) bounds them on both sides
+  if (p.wr >= 0) {
     const int i_max = min(U.q_len - 1, (U.row0 + NQ * kBM - 1) / p.P);
-    hi = min(hi, (long long)i_max + U.delta + 1);
+    hi = min(hi, (long long)i_max + U.delta + p.wr + 1);
+  }
+  if (p.wl >= 0) {
+    const int i_min = U.row0 / p.P;
+    lo = max(lo, (long long)i_min + U.delta - p.wl);
   }
   U.kv_lo = (int)lo;
   U.kv_hi = (int)max(hi, lo);
@@ -297,10 +321,14 @@ __host__ __device__ constexpr uint32_t instr_desc(int M, int N, bool a_mn_major,
          | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-template <int D_, int BN_, int NQ_, int NS_, int KST_, int VST_, bool HALF_, bool PARTIAL_>
+template <int D_, int BN_, int NQ_, int NS_, int KST_, int VST_, bool HALF_, bool PARTIAL_,
+          bool MODS_ = false>
 struct FwdCfg {
   static constexpr int D = D_, BN = BN_, NQ = NQ_, NS = NS_, KST = KST_, VST = VST_;
   static constexpr bool HALF = HALF_, PARTIAL = PARTIAL_;
+  // score/mask modifiers beyond causal (left window bound, soft-cap): a
+  // separate kernel, so that the plain one carries none of their cost
+  static constexpr bool MODS = MODS_;
   static constexpr int kChunks = D / 64;          // 128-byte column chunks of a row
   static constexpr int kQTile = kBM * D * 2;      // bytes
   static constexpr int kKVTile = BN * D * 2;
@@ -827,7 +855,9 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
     const int nb = U.nb;
     // per-row constants relative to the unit's first key kv_lo, so that the
     // unit record can die before the KV loop
-    const int lim_rel = (p.causal ? min(U.kv_hi, i + U.delta + 1) : U.kv_hi) - U.kv_lo;
+    // admitted keys of this row, relative to kv_lo: [st_rel, lim_rel)
+    const int lim_rel = (p.wr >= 0 ? min(U.kv_hi, i + U.delta + p.wr + 1) : U.kv_hi) - U.kv_lo;
+    const int st_rel = (C::MODS && p.wl >= 0) ? max(0, i + U.delta - p.wl - U.kv_lo) : 0;
     const int base0 = i + U.delta - U.kv_lo;  // distance of column 0 of tile 0
     const size_t orow = (size_t)(U.q_start + i) * p.Hq + h;  // packed (token, head) row
     void *out_row;
@@ -856,9 +886,10 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
                                                         base - (BN - 1) < p.R);
       const uint32_t s_addr = tmem + lane_addr + C::s_col(t, buf);
       const int lim_c = lim_rel - jrel;  // columns at or past lim_c are masked
+      const int st_c = C::MODS ? st_rel - jrel : 0;  // and columns before st_c
       // no row of the warp has a masked column here: the FMA-pipe exponential
       // may stand in for some of the MUFU ones
-      const bool poly_ok = __all_sync(0xffffffffu, lim_c >= BN);
+      const bool poly_ok = __all_sync(0xffffffffu, lim_c >= BN && st_c <= 0);
       // one arrival per warp, after this thread's tensor-memory accesses
       auto warp_arrive = [&](int b) {
         tc_fence_before();
@@ -933,16 +964,19 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
             }
             // every score read: the next tile's upper keys may land
             if (C::kSplitS && hf == BN / 64 - 1) warp_arrive(C::bSRead + t);
+            if constexpr (C::MODS) {
+              if (p.cap_a > 0.f) softcap_all<64>(x, p.cap_a, p.cap_b);
+            }
             if (bon) bias_apply<C::HALF>(bv, bsh, p.inv_scale, x);
             if (hf + 1 < BN / 64) {
               const int lo = lo0 - 64 * (hf + 1);
               bon = half_on(lo);
               if (bon) bias_fetch(brow, lo, p.R, bv);
             }
-            if (lim_c < 64 * hf + 64) {
+            if (lim_c < 64 * hf + 64 || st_c > 64 * hf) {
 #pragma unroll
               for (int e = 0; e < 64; ++e)
-                if (64 * hf + e >= lim_c) x[e] = -INFINITY;
+                if (64 * hf + e >= lim_c || 64 * hf + e < st_c) x[e] = -INFINITY;
             }
           // running-max update with conditional rescaling
           const float m_new = fmaxf(m_ref, row_max<0, 64>(x));
@@ -1010,10 +1044,13 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
           }
           tmem_wait_ld();
           if (C::kSplitS) warp_arrive(C::bSRead + t);
-          if (lim_c < BN) {
+          if constexpr (C::MODS) {
+            if (p.cap_a > 0.f) softcap_all<BN>(s, p.cap_a, p.cap_b);
+          }
+          if (lim_c < BN || st_c > 0) {
 #pragma unroll
             for (int c = 0; c < BN; ++c)
-              if (c >= lim_c) s[c] = -INFINITY;
+              if (c >= lim_c || c < st_c) s[c] = -INFINITY;
           }
           const float m_new = fmaxf(m_ref, row_max<0, BN>(s));
           if (n == 0) {

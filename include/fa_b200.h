@@ -163,6 +163,54 @@ fa_status fa_fwd_splitkv_static(const void *q, const void *k, const void *v,
                                 int rel_extent, int num_splits, void *stream);
 
 /*
+ * Score and mask modifiers ("mgoin/tml-fa4" lists mask/score modifiers among
+ * the forward paths; the two below are the plain readings this library
+ * serves).  With d = i + (k_len - q_len) - j the distance of key j from query
+ * row i's diagonal (the distance of the causal and bias rules):
+ *   window_left  >= 0: key j is masked when d > window_left (more than
+ *                 window_left keys before the diagonal); < 0: no bound.
+ *   window_right >= 0: key j is masked when -d > window_right (more than
+ *                 window_right keys after the diagonal); < 0: no bound.
+ *                 causal mode is window_right = 0 (a larger value is capped).
+ *   softcap      >  0: the scaled score s becomes softcap * tanh(s / softcap)
+ *                 before rel_bias is added; 0: off.  Must be finite, >= 0.
+ * A row whose window holds no key gets O = 0 and LSE = -inf.  Keys outside
+ * the window are neither loaded nor multiplied when they fill whole key
+ * tiles.  FA_MODS_NONE initialises a struct with no modifier; a NULL pointer
+ * means the same.
+ */
+typedef struct {
+  int window_left;
+  int window_right;
+  float softcap;
+} fa_mods;
+#define FA_MODS_NONE {-1, -1, 0.0f}
+
+/* fa_fwd, fa_fwd_varlen and fa_fwd_splitkv with modifiers (`mods` may be
+ * NULL; it is read during the call only). */
+fa_status fa_fwd_ex(const void *q, const void *k, const void *v, void *out,
+                    float *lse, int B, int Sq, int Sk, int Hq, int Hkv, int D,
+                    fa_dtype dt, int causal, float softmax_scale,
+                    const int *seqused_k, const void *rel_bias, int rel_extent,
+                    const fa_mods *mods, void *stream);
+fa_status fa_fwd_varlen_ex(const void *q, const void *k, const void *v,
+                           void *out, float *lse, const int *cu_seqlens_q,
+                           const int *cu_seqlens_k, const int *seqused_k,
+                           int B, int max_seqlen_q, int max_seqlen_k,
+                           int total_q, int total_k, int Hq, int Hkv, int D,
+                           fa_dtype dt, int causal, float softmax_scale,
+                           const void *rel_bias, int rel_extent,
+                           const fa_mods *mods, void *stream);
+fa_status fa_fwd_splitkv_ex(const void *q, const void *k, const void *v,
+                            void *out, float *lse, int B, int Sq, int Sk,
+                            int Hq, int Hkv, int D, fa_dtype dt, int causal,
+                            float softmax_scale, const int *seqused_k,
+                            const void *rel_bias, int rel_extent,
+                            int num_splits, void *workspace,
+                            size_t workspace_bytes, const fa_mods *mods,
+                            void *stream);
+
+/*
  * Device-side watchdog.  Every wait inside the kernels is bounded; a kernel
  * that gives up records a code in a device word and returns without
  * trapping.  This call synchronises the current device, copies that word to

@@ -68,6 +68,12 @@ def test_validation_statuses(lib):
     assert _fwd(lib, rb=A, R=0) == FA_ERR_INVALID
     assert _fwd(lib, rb=MIS, R=128) == FA_ERR_INVALID
     assert _fwd(lib, scale=float("nan")) == FA_ERR_INVALID
+    import exact_attention_forward_flash_b200 as fa
+    for bad in (float("nan"), -1.0, float("inf")):
+        m = fa.FaMods(-1, -1, bad)
+        r = lib.fa_fwd_ex(A, A, A, A, A, 1, 16, 16, 4, 2, 128, 0, 0, 0.0, None, None, 0,
+                          ctypes.byref(m), None)
+        assert r == FA_ERR_INVALID, bad
     assert _fwd(lib, Sq=-1) == FA_ERR_INVALID
     assert _fwd(lib, B=-1) == FA_ERR_INVALID
     msg = lib.fa_last_error_message().decode()

@@ -36,26 +36,27 @@ def run_dense(p, **kw):
     return out, lse
 
 
-def ref_dense(p):
+def ref_dense(p, window=(-1, -1), softcap=0.0):
     return oracle.attention(p.q, p.k, p.v, causal=p.causal, softmax_scale=p.softmax_scale,
-                            seqused_k=p.seqused_k, rel_bias=p.rel_bias)
+                            seqused_k=p.seqused_k, rel_bias=p.rel_bias, window=window,
+                            softcap=softcap)
 
 
-def run_varlen(p):
+def run_varlen(p, **kw):
     g = p.to(DEV)
     out, lse = fa.fa_fwd_varlen(g.q, g.k, g.v, g.cu_seqlens_q, g.cu_seqlens_k,
                                 p.max_seqlen_q, p.max_seqlen_k, seqused_k=g.seqused_k,
                                 causal=p.causal, softmax_scale=p.softmax_scale,
-                                rel_bias=g.rel_bias)
+                                rel_bias=g.rel_bias, **kw)
     torch.cuda.synchronize()
     return out, lse
 
 
-def ref_varlen(p):
+def ref_varlen(p, window=(-1, -1), softcap=0.0):
     return oracle.attention(p.q, p.k, p.v, cu_seqlens_q=p.cu_seqlens_q,
                             cu_seqlens_k=p.cu_seqlens_k, seqused_k=p.seqused_k,
                             causal=p.causal, softmax_scale=p.softmax_scale,
-                            rel_bias=p.rel_bias)
+                            rel_bias=p.rel_bias, window=window, softcap=softcap)
 
 
 # ---------------------------------------------------------------------------
@@ -336,3 +337,65 @@ def test_invalid_arguments_raise_and_write_nothing():
         fa.fa_fwd(q, k, k, out=out)
     torch.cuda.synchronize()
     assert (out == 7.0).all()
+
+
+
+# ---------------------------------------------------------------------------
+# score and mask modifiers: sliding window, soft-cap (fa_mods)
+# ---------------------------------------------------------------------------
+WINDOW_CASES = [
+    # B, Sq, Sk, Hq, Hkv, D, causal, (left, right)
+    (2, 700, 700, 4, 2, 128, True, (200, -1)),    # causal sliding window
+    (1, 500, 900, 8, 2, 128, False, (128, 64)),   # two-sided, k longer
+    (1, 900, 400, 4, 4, 128, False, (-1, 0)),     # right bound only = causal
+    (1, 300, 300, 8, 1, 256, True, (63, -1)),     # D = 256
+    (2, 400, 650, 4, 2, 64, False, (300, 10)),    # D = 64
+    (1, 260, 100, 4, 4, 128, False, (0, 0)),      # diagonal key only; early rows see none
+]
+
+
+@pytest.mark.parametrize("case", WINDOW_CASES)
+def test_window(case):
+    B, Sq, Sk, Hq, Hkv, D, causal, win = case
+    p = fa_inputs.random_dense(200 + Sq + Sk, B, Sq, Sk, Hq, Hkv, D, causal=causal)
+    out, lse = run_dense(p, window=win)
+    ro, rl = ref_dense(p, window=win)
+    compare(out, lse, ro, rl, what=f"window {case}")
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+def test_softcap(D, causal):
+    # q sharpened so that the cap matters (scaled scores well beyond it)
+    p = fa_inputs.random_dense(300 + D, 2, 333, 410, 8, 2, D, causal=causal, q_std=4.0)
+    out, lse = run_dense(p, softcap=5.0)
+    ro, rl = ref_dense(p, softcap=5.0)
+    compare(out, lse, ro, rl, what=f"softcap D{D} causal={causal}")
+
+
+@pytest.mark.parametrize("D", [128, 256])
+def test_varlen_window_softcap_bias(D):
+    q_lens = [0, 1, 130, 513, 257, 64]
+    k_lens = [3, 1, 200, 513, 300, 0]
+    p = fa_inputs.random_varlen(41 + D, q_lens, k_lens, Hq=8, Hkv=2, D=D, causal=True,
+                                bias_extent=256)
+    out, lse = run_varlen(p, window=(150, -1), softcap=10.0)
+    ro, rl = ref_varlen(p, window=(150, -1), softcap=10.0)
+    compare(out, lse, ro, rl, what=f"varlen window+softcap+bias D{D}")
+
+
+def test_splitkv_window_softcap():
+    p = fa_inputs.random_dense(51, 3, 2, 3000, 8, 2, 128, q_std=3.0)
+    g = p.to(DEV)
+    out, lse = fa.fa_fwd_splitkv(g.q, g.k, g.v, num_splits=5, window=(1200, -1), softcap=8.0)
+    torch.cuda.synchronize()
+    ro, rl = ref_dense(p, window=(1200, -1), softcap=8.0)
+    compare(out, lse, ro, rl, what="splitkv window+softcap")
+
+
+def test_window_off_matches_no_modifiers():
+    # the window encoding of "no bound" gives bit-identical results
+    p = fa_inputs.random_dense(61, 1, 300, 300, 4, 2, 128, causal=True)
+    a, la = run_dense(p)
+    b, lb = run_dense(p, window=(-1, -1), softcap=0.0)
+    assert torch.equal(a, b) and torch.equal(la, lb)
