@@ -36,7 +36,8 @@ if ROOT not in sys.path:
 
 METRIC = "attention fwd TFLOP/s & % of BF16 tensor peak; split-KV decode HBM GB/s"
 MAIN = "varlen_gqa_bias"
-EXTRAS = ["dense_257", "video_dit_20480", "encoder_d256_seqused", "decode_splitkv", "dense_d64"]
+EXTRAS = ["dense_257", "video_dit_20480", "encoder_d256_seqused", "decode_splitkv", "dense_d64",
+          "local_window_softcap"]
 DESCR = {
     "dense_257": "dense non-causal MHA B=1 S=257 H=8 D=128 bf16",
     "varlen_gqa_bias": "varlen causal GQA 32/8 D=128, 4 seqs U[512,4096] (seeded), rel_bias R=256 bf16",
@@ -44,6 +45,7 @@ DESCR = {
     "encoder_d256_seqused": "dense GQA 8/1 D=256 B=2 Sq=1024 Sk=1024 seqused_k=968 bf16",
     "decode_splitkv": "split-KV decode B=8 Sq=1 Sk=131072 Hq=32 Hkv=8 D=128 bf16",
     "dense_d64": "dense non-causal MHA B=4 S=4096 H=16 D=64 bf16",
+    "local_window_softcap": "causal GQA 16/4 D=128 B=1 S=32768, window 4095 left, softcap 50 bf16",
 }
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
 
@@ -211,16 +213,18 @@ class Runner:
         if p.splitkv:
             fa.fa_fwd_splitkv(q, k, v, num_splits=self.ns, causal=p.causal,
                               softmax_scale=p.softmax_scale, seqused_k=p.seqused_k,
-                              rel_bias=rb, out=self.out, lse=self.lse, workspace=self.ws)
+                              rel_bias=rb, out=self.out, lse=self.lse, workspace=self.ws,
+                              window=p.window, softcap=p.softcap)
         elif p.layout == "dense":
             fa.fa_fwd(q, k, v, causal=p.causal, softmax_scale=p.softmax_scale,
-                      seqused_k=p.seqused_k, rel_bias=rb, out=self.out, lse=self.lse)
+                      seqused_k=p.seqused_k, rel_bias=rb, out=self.out, lse=self.lse,
+                      window=p.window, softcap=p.softcap)
         else:
             cq, ck = (p.cu_seqlens_q, p.cu_seqlens_k) if cu is None else cu
             fa.fa_fwd_varlen(q, k, v, cq, ck, p.max_seqlen_q, p.max_seqlen_k,
                              seqused_k=p.seqused_k, causal=p.causal,
                              softmax_scale=p.softmax_scale, rel_bias=rb, out=self.out,
-                             lse=self.lse)
+                             lse=self.lse, window=p.window, softcap=p.softcap)
 
 
 def time_steps(step, steps: int, warmup: int, dist_on: bool, device_index: int,
@@ -316,8 +320,7 @@ def oracle_rows_sample(p, n_rows: int, seed: int = 0):
             ql, kl = lens[b]
         i = int(rng.integers(ql))
         h = int(rng.integers(p.Hq))
-        keys = min(kl, i + (kl - ql) + 1) if p.causal else kl
-        flops += 4.0 * p.D * max(keys, 0)
+        flops += 4.0 * p.D * p.admitted_keys(ql, kl, i)
         rows.append((b, h, i))
     return np.array(rows, dtype=np.int32), flops
 
@@ -325,7 +328,8 @@ def oracle_rows_sample(p, n_rows: int, seed: int = 0):
 def time_oracle(p_cpu, target_s: float):
     import oracle
     kw = dict(causal=p_cpu.causal, softmax_scale=p_cpu.softmax_scale,
-              seqused_k=p_cpu.seqused_k, rel_bias=p_cpu.rel_bias)
+              seqused_k=p_cpu.seqused_k, rel_bias=p_cpu.rel_bias, window=p_cpu.window,
+              softcap=p_cpu.softcap)
     if p_cpu.layout == "varlen":
         kw.update(cu_seqlens_q=p_cpu.cu_seqlens_q, cu_seqlens_k=p_cpu.cu_seqlens_k)
     n = 64
@@ -505,7 +509,7 @@ def run_reference(a, world):
     # size one step to ~cpu_seconds / steps of CPU work
     v0, secs0, n0 = time_oracle(p, max(0.5, a.cpu_seconds / max(1, a.steps + a.warmup)))
     kw = dict(causal=p.causal, softmax_scale=p.softmax_scale, seqused_k=p.seqused_k,
-              rel_bias=p.rel_bias)
+              rel_bias=p.rel_bias, window=p.window, softcap=p.softcap)
     if p.layout == "varlen":
         kw.update(cu_seqlens_q=p.cu_seqlens_q, cu_seqlens_k=p.cu_seqlens_k)
     samples = [oracle_rows_sample(p, n0, seed=s) for s in range(a.warmup + a.steps)]

@@ -21,6 +21,9 @@ Workloads (shapes from the pages' validation tables and API contracts):
   decode with an LSE combine.
 * ``dense_d64``: dense non-causal MHA, B=4, S=4096, H=16, D=64 (a 64-wide
   head dim, one of the small head dims the pages list as the next step).
+* ``local_window_softcap``: causal GQA 16/4, D=128, B=1, S=32768 with a
+  sliding window of 4095 keys to the left and scores soft-capped at 50 (the
+  pages' "mask/score modifiers", at local-attention sizes).
 
 Seeds are 440410 + workload index (the seed style of the pages' benchmark).
 Values are drawn in float32 as N(0, 1) and rounded to the input dtype.
@@ -36,7 +39,8 @@ import torch
 SEED_BASE = 440410
 
 WORKLOADS = ["dense_257", "varlen_gqa_bias", "video_dit_20480",
-             "encoder_d256_seqused", "decode_splitkv", "dense_d64"]
+             "encoder_d256_seqused", "decode_splitkv", "dense_d64",
+             "local_window_softcap"]
 
 _CHUNK = 1 << 24
 
@@ -75,6 +79,8 @@ class Problem:
     max_seqlen_k: int = 0
     splitkv: bool = False
     meta: dict = field(default_factory=dict)
+    window: tuple = (-1, -1)         # (left, right) bounds by diagonal distance; < 0: none
+    softcap: float = 0.0             # > 0: scores capped as softcap * tanh(s / softcap)
 
     # -- shapes -----------------------------------------------------------
     @property
@@ -111,9 +117,28 @@ class Problem:
         return lens
 
     # -- algorithmic work (the metric's definition) ------------------------
+    def admitted_keys(self, ql: int, kl: int, i: int) -> int:
+        """Keys row i of a (q_len, k_len) sequence attends to under the
+        causal flag and the window (distance d = i + kl - ql - j)."""
+        delta = kl - ql
+        lo, hi = 0, kl - 1
+        wl, wr = self.window
+        if self.causal:
+            wr = 0 if wr < 0 else min(wr, 0)
+        if wr >= 0:
+            hi = min(hi, i + delta + wr)
+        if wl >= 0:
+            lo = max(lo, i + delta - wl)
+        return max(0, hi - lo + 1)
+
     def flops(self) -> float:
-        """4 * q_len * k_len * D * Hq per sequence, halved when causal."""
+        """4 * q_len * k_len * D * Hq per sequence, halved when causal; with a
+        window, 4 * D * Hq per admitted (row, key) pair."""
         f = 0.0
+        if self.window[0] >= 0 or self.window[1] >= 0:
+            for ql, kl in self.seq_lens():
+                f += 4.0 * self.D * self.Hq * sum(self.admitted_keys(ql, kl, i) for i in range(ql))
+            return f
         for ql, kl in self.seq_lens():
             f += 4.0 * ql * kl * self.D * self.Hq
         return f * (0.5 if self.causal else 1.0)
@@ -141,7 +166,7 @@ class Problem:
                        self.causal, self.softmax_scale, kw["cu_seqlens_q"],
                        kw["cu_seqlens_k"], kw["seqused_k"], kw["rel_bias"],
                        self.max_seqlen_q, self.max_seqlen_k, self.splitkv,
-                       dict(self.meta))
+                       dict(self.meta), tuple(self.window), self.softcap)
 
 
 def make(name: str, dtype=torch.bfloat16, device="cpu", decode_sk: int = 131072) -> Problem:
@@ -206,6 +231,13 @@ def make(name: str, dtype=torch.bfloat16, device="cpu", decode_sk: int = 131072)
         v = _randn((B, S, H, D), g, dtype)
         return Problem(name, "dense", q, k, v, softmax_scale=1 / math.sqrt(D),
                        max_seqlen_q=S, max_seqlen_k=S)
+    if name == "local_window_softcap":
+        B, S, Hq, Hkv, D = 1, 32768, 16, 4, 128
+        q = _randn((B, S, Hq, D), g, dtype)
+        k = _randn((B, S, Hkv, D), g, dtype)
+        v = _randn((B, S, Hkv, D), g, dtype)
+        return Problem(name, "dense", q, k, v, causal=True, softmax_scale=1 / math.sqrt(D),
+                       max_seqlen_q=S, max_seqlen_k=S, window=(4095, -1), softcap=50.0)
     raise KeyError(name)
 
 

@@ -399,3 +399,16 @@ def test_window_off_matches_no_modifiers():
     a, la = run_dense(p)
     b, lb = run_dense(p, window=(-1, -1), softcap=0.0)
     assert torch.equal(a, b) and torch.equal(la, lb)
+
+
+def test_local_window_softcap_workload_sampled():
+    p = fa_inputs.make("local_window_softcap")
+    out, lse = run_dense(p, window=p.window, softcap=p.softcap)
+    rows = _sample_rows(np.random.default_rng(3), 1, 16, [32768], 256)
+    ro, rl = oracle.attention_rows(p.q, p.k, p.v, rows, softmax_scale=p.softmax_scale,
+                                   causal=True, window=p.window, softcap=p.softcap)
+    o = out.float().cpu()
+    l = lse.cpu()
+    go = np.stack([o[b, i, h].numpy() for b, h, i in rows])
+    gl = np.array([float(l[b, h, i]) for b, h, i in rows])
+    compare(go, gl, ro, rl, what="local_window_softcap sampled")
