@@ -92,6 +92,8 @@ def load_library(path: Optional[str] = None):
     lib.fa_fwd_varlen_ex.restype = i32
     lib.fa_fwd_splitkv_ex.argtypes = lib.fa_fwd_splitkv.argtypes[:-1] + [M, P]
     lib.fa_fwd_splitkv_ex.restype = i32
+    lib.fa_watchdog_selftest.argtypes = [ctypes.c_ulonglong, P]
+    lib.fa_watchdog_selftest.restype = i32
     lib.fa_check_device_error.argtypes = [ctypes.POINTER(i32), i32]
     lib.fa_check_device_error.restype = i32
     lib.fa_status_string.argtypes = [i32]
@@ -301,6 +303,11 @@ def check_device_error(clear: bool = True) -> int:
     if st not in (FA_OK, 5):
         _check(st)
     return int(code.value)
+
+
+def watchdog_selftest(timeout_s: float = 0.05, stream=None) -> None:
+    """Enqueue the watchdog self-test (a bounded wait that must time out)."""
+    _check(load_library().fa_watchdog_selftest(int(timeout_s * 1e9), _stream(stream)))
 
 
 def version() -> str:

@@ -484,6 +484,16 @@ fa_status fa_fwd_splitkv_ex(const void *q, const void *k, const void *v, void *o
                                            B * Sq, 1, st);
 }
 
+fa_status fa_watchdog_selftest(unsigned long long timeout_ns, void *stream) {
+  g_msg[0] = 0;
+  if (timeout_ns < 1000000ull || timeout_ns > 1000000000ull)
+    return fail(FA_ERR_INVALID, "timeout_ns must be within [1 ms, 1 s]");
+  fab::fa_watchdog_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "self-test launch: %s", cudaGetErrorString(e));
+  return FA_OK;
+}
+
 fa_status fa_check_device_error(int *code, int clear) {
   unsigned v = 0;
   cudaError_t e = cudaDeviceSynchronize();

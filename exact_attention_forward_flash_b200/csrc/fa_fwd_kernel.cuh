@@ -1219,6 +1219,21 @@ __global__ void __launch_bounds__(C::kThreads, 1) fa_fwd_kernel(const __grid_con
 }
 
 // ---------------------------------------------------------------------------
+// watchdog self-test: one thread waits, bounded by timeout_ns, on a fresh
+// mbarrier that nothing ever arrives at, so the wait must give up, record the
+// timeout code in the watchdog word and return (no trap, no endless loop).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(32) fa_watchdog_selftest_kernel(unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) (void)mbar_wait(smem_u32(&bar), 0u, &g_fa_error, timeout_ns);
+}
+
+// ---------------------------------------------------------------------------
 // split-KV merge: one warp per packed (token, head) row
 // ---------------------------------------------------------------------------
 template <int D, bool HALF>

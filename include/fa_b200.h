@@ -60,7 +60,7 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID = 1,        /* malformed arguments (null, shape, alignment) */
-  FA_ERR_UNSUPPORTED = 2,    /* well-formed but not served (e.g. D = 64)    */
+  FA_ERR_UNSUPPORTED = 2,    /* well-formed but not served (e.g. D = 96)    */
   FA_ERR_CUDA = 3,           /* a CUDA runtime call or launch failed         */
   FA_ERR_WORKSPACE = 4,      /* split-KV workspace missing or too small      */
   FA_ERR_DEVICE_TIMEOUT = 5  /* a kernel gave up waiting (see below)         */
@@ -218,6 +218,16 @@ fa_status fa_fwd_splitkv_ex(const void *q, const void *k, const void *v,
  * FA_ERR_DEVICE_TIMEOUT when the word was set, or FA_ERR_CUDA.
  */
 fa_status fa_check_device_error(int *code, int clear);
+
+/*
+ * Watchdog self-test: enqueues one thread that waits, bounded by timeout_ns
+ * (1 ms to 1 s), on a barrier nothing ever completes.  The wait gives up and
+ * records the timeout code in the watchdog word exactly as a stalled kernel
+ * would, without trapping; the device stays usable.  A following
+ * fa_check_device_error then returns FA_ERR_DEVICE_TIMEOUT (and clears the
+ * word when asked).  Returns FA_OK once enqueued.
+ */
+fa_status fa_watchdog_selftest(unsigned long long timeout_ns, void *stream);
 
 /* Human-readable name of a status; never NULL. */
 const char *fa_status_string(fa_status s);

@@ -117,3 +117,9 @@ def test_status_strings(lib):
     for s, name in [(0, "FA_OK"), (1, "FA_ERR_INVALID"), (2, "FA_ERR_UNSUPPORTED"),
                     (3, "FA_ERR_CUDA"), (4, "FA_ERR_WORKSPACE"), (5, "FA_ERR_DEVICE_TIMEOUT")]:
         assert lib.fa_status_string(s).decode() == name
+
+
+def test_watchdog_selftest_validates_its_limit(lib):
+    # out of [1 ms, 1 s]: rejected before anything is enqueued
+    assert lib.fa_watchdog_selftest(10, None) == FA_ERR_INVALID
+    assert lib.fa_watchdog_selftest(5_000_000_000, None) == FA_ERR_INVALID

@@ -412,3 +412,16 @@ def test_local_window_softcap_workload_sampled():
     go = np.stack([o[b, i, h].numpy() for b, h, i in rows])
     gl = np.array([float(l[b, h, i]) for b, h, i in rows])
     compare(go, gl, ro, rl, what="local_window_softcap sampled")
+
+
+def test_watchdog_timeout_is_reported_and_the_device_stays_usable():
+    # a bounded wait that nothing completes must give up, record the timeout
+    # code (1) and leave the context usable
+    assert fa.check_device_error() == 0
+    fa.watchdog_selftest(0.05)
+    assert fa.check_device_error(clear=True) == 1
+    assert fa.check_device_error() == 0
+    p = fa_inputs.random_dense(71, 1, 130, 200, 4, 2, 128, causal=True)
+    out, lse = run_dense(p)
+    ro, rl = ref_dense(p)
+    compare(out, lse, ro, rl, what="after the watchdog self-test")
