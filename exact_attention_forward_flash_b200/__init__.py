@@ -92,6 +92,11 @@ def load_library(path: Optional[str] = None):
     lib.fa_fwd_varlen_ex.restype = i32
     lib.fa_fwd_splitkv_ex.argtypes = lib.fa_fwd_splitkv.argtypes[:-1] + [M, P]
     lib.fa_fwd_splitkv_ex.restype = i32
+    lib.fa_fwd_shard_partial.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32,
+                                         i32, f32, P, P, P, i32, M, i32, P, ctypes.c_size_t, P]
+    lib.fa_fwd_shard_partial.restype = i32
+    lib.fa_combine_partials.argtypes = [P, P, i32, i32, i32, i32, i32, i32, P, P, P]
+    lib.fa_combine_partials.restype = i32
     lib.fa_watchdog_selftest.argtypes = [ctypes.c_ulonglong, P]
     lib.fa_watchdog_selftest.restype = i32
     lib.fa_check_device_error.argtypes = [ctypes.POINTER(i32), i32]
@@ -264,6 +269,78 @@ def fa_fwd_splitkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
         _ptr(seqused_k), _ptr(rel_bias), R, int(ns), _ptr(workspace),
         workspace.numel() * workspace.element_size(), ctypes.byref(m),
         _stream(stream)))
+    return out, lse
+
+
+def fa_fwd_shard_partial(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
+                         k_after: Optional[torch.Tensor] = None,
+                         causal: bool = False, softmax_scale: Optional[float] = None,
+                         seqused_k: Optional[torch.Tensor] = None,
+                         rel_bias: Optional[torch.Tensor] = None,
+                         window: Optional[Tuple[int, int]] = None, softcap: float = 0.0,
+                         num_splits: int = 1,
+                         o_part: Optional[torch.Tensor] = None,
+                         lse_part: Optional[torch.Tensor] = None,
+                         workspace: Optional[torch.Tensor] = None,
+                         stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Normalised fp32 partial of one key shard: q [B,Sq,Hq,D] (all query
+    rows), k/v [B,Sk,Hkv,D] (this shard's keys), k_after int32 [B] (keys of
+    each sequence after the shard).  Returns (o_part [B*Sq*Hq, D] fp32,
+    lse_part [B*Sq*Hq] fp32), packed (token, head) rows."""
+    lib = load_library()
+    B, Sq, Hq, D = q.shape
+    _, Sk, Hkv, _ = k.shape
+    rows = B * Sq * Hq
+    if o_part is None:
+        o_part = torch.empty((rows, D), dtype=torch.float32, device=q.device)
+    if lse_part is None:
+        lse_part = torch.empty((rows,), dtype=torch.float32, device=q.device)
+    ns = num_splits
+    if ns <= 0:
+        ns = splitkv_default_splits(B, Sq, max(Sk, 1), Hq, Hkv, D,
+                                    torch.cuda.get_device_properties(q.device).multi_processor_count)
+    if workspace is None and ns > 1:
+        workspace = torch.empty(max(splitkv_workspace_bytes(B, Sq, Hq, D, ns), 16),
+                                dtype=torch.uint8, device=q.device)
+    _need_cuda(q, k, v, o_part, lse_part, seqused_k, k_after, rel_bias, workspace)
+    _same_dtype(q, k, v, rel_bias)
+    for t, n in ((o_part, "o_part"), (lse_part, "lse_part")):
+        if t.dtype != torch.float32 or not t.is_contiguous():
+            raise TypeError(f"{n} must be a contiguous float32 tensor")
+    _int32(seqused_k, "seqused_k")
+    _int32(k_after, "k_after")
+    R = 0 if rel_bias is None else int(rel_bias.shape[-1])
+    m = _mods(window, softcap)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.fa_fwd_shard_partial(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o_part), _ptr(lse_part), B, Sq, Sk, Hq, Hkv, D,
+        _dtype(q), int(bool(causal)), float(softmax_scale or 0.0), _ptr(seqused_k),
+        _ptr(k_after), _ptr(rel_bias), R, ctypes.byref(m), int(ns), _ptr(workspace),
+        ws_bytes, _stream(stream)))
+    return o_part, lse_part
+
+
+def fa_combine_partials(o_parts: torch.Tensor, lse_parts: torch.Tensor, B: int, Sq: int,
+                        Hq: int, *, dtype: torch.dtype = torch.bfloat16,
+                        out: Optional[torch.Tensor] = None,
+                        lse: Optional[torch.Tensor] = None,
+                        stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Merge stacked partials o_parts [n, B*Sq*Hq, D] / lse_parts [n, B*Sq*Hq]
+    into (out [B,Sq,Hq,D] of `dtype`, lse [B,Hq,Sq])."""
+    lib = load_library()
+    n, rows, D = o_parts.shape
+    if rows != B * Sq * Hq or tuple(lse_parts.shape) != (n, rows):
+        raise ValueError("o_parts must be [n, B*Sq*Hq, D] and lse_parts [n, B*Sq*Hq]")
+    if out is None:
+        out = torch.empty((B, Sq, Hq, D), dtype=dtype, device=o_parts.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=o_parts.device)
+    _need_cuda(o_parts, lse_parts, out, lse)
+    for t, nm in ((o_parts, "o_parts"), (lse_parts, "lse_parts")):
+        if t.dtype != torch.float32 or not t.is_contiguous():
+            raise TypeError(f"{nm} must be a contiguous float32 tensor")
+    _check(lib.fa_combine_partials(_ptr(o_parts), _ptr(lse_parts), n, B, Sq, Hq, D,
+                                   _dtype(out), _ptr(out), _ptr(lse), _stream(stream)))
     return out, lse
 
 

@@ -185,6 +185,8 @@ struct Common {
   // modifiers (fa_mods): window bounds (< 0: none), soft-cap (0: off)
   int window_left = -1, window_right = -1;
   float softcap = 0.f;
+  // key shard: per-batch count of the sequence's keys after the ones given
+  const int *k_after = nullptr;
 };
 
 void apply_mods(Common &c, const fa_mods *m) {
@@ -258,6 +260,7 @@ fa_status fill_params(const Common &c, FwdParams &p, int nq, int bn, int num_spl
   p.cu_q = c.varlen ? c.cu_q : nullptr;
   p.cu_k = c.varlen ? c.cu_k : nullptr;
   p.seqused_k = c.seqused_k;
+  p.k_after = c.k_after;
   p.rel_bias = static_cast<const uint16_t *>(c.rel_bias);
   p.R = c.rel_bias ? c.R : 0;
   p.B = c.B;
@@ -315,21 +318,95 @@ fa_status run_fwd(const Common &c, cudaStream_t st) {
   return launch_variant<Fwd256>(p, dev, st, half, mods);
 }
 
-template <int D, bool HALF>
+template <int D, bool HALF, bool F32OUT>
 fa_status launch_combine(const float *o_part, const float *lse_part, int ns, long long rows,
                          void *out, float *lse, int Hq, int Sq, int total_q, int lse_dense,
                          cudaStream_t st) {
   const int warps = 8;
   const long long blocks = (rows + warps - 1) / warps;
   if (blocks > 0x7fffffffLL) return fail(FA_ERR_UNSUPPORTED, "too many rows");
-  fa_combine_kernel<D, HALF><<<(unsigned)blocks, warps * 32, 0, st>>>(
+  fa_combine_kernel<D, HALF, F32OUT><<<(unsigned)blocks, warps * 32, 0, st>>>(
       o_part, lse_part, ns, rows, out, lse, Hq, Sq, total_q, lse_dense);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(FA_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
   return FA_OK;
 }
 
+// Merge ns partials of `rows` packed rows of a dense [B, Sq, Hq] problem:
+// into out (input dtype) and lse [B, Hq, Sq], or, with f32out, into one
+// fp32 partial (out [rows][D], lse [rows]).
+fa_status combine(int D, bool half, bool f32out, const float *o_part, const float *lse_part,
+                  int ns, long long rows, void *out, float *lse, int Hq, int Sq, int B,
+                  cudaStream_t st) {
+  const int tq = B * Sq;
+#define FA_COMBINE(DD)                                                                      \
+  if (f32out)                                                                               \
+    return launch_combine<DD, false, true>(o_part, lse_part, ns, rows, out, lse, Hq, Sq, tq, \
+                                           1, st);                                          \
+  return half ? launch_combine<DD, true, false>(o_part, lse_part, ns, rows, out, lse, Hq, Sq, \
+                                                tq, 1, st)                                   \
+              : launch_combine<DD, false, false>(o_part, lse_part, ns, rows, out, lse, Hq,  \
+                                                 Sq, tq, 1, st);
+  if (D == 64) { FA_COMBINE(64) }
+  if (D == 128) { FA_COMBINE(128) }
+  FA_COMBINE(256)
+#undef FA_COMBINE
+}
+
 int splitkv_bn(int D) { return D == 256 ? 64 : 128; }
+
+
+// Split-KV forward of a dense problem: the keys are cut into num_splits
+// ranges whose normalised fp32 partials go to the workspace and are merged
+// by LSE into c.out / c.lse, or, with to_partial, into one fp32 partial
+// (c.out as float [B*Sq*Hq][D], c.lse as float [B*Sq*Hq]).  A single split
+// writes a partial in place and needs no workspace.
+fa_status run_splitkv(const Common &c, int num_splits, void *workspace, size_t workspace_bytes,
+                      bool to_partial, cudaStream_t st) {
+  fa_status s = validate(c);
+  if (s != FA_OK) return s;
+  if (num_splits < 0) return fail(FA_ERR_INVALID, "num_splits must be >= 0");
+  const int B = c.B, Sq = c.Sq, Sk = c.Sk, Hq = c.Hq, D = c.D;
+  if ((long long)B * Sq == 0) return FA_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(FA_ERR_CUDA, "cudaGetDevice failed");
+  if (Sk == 0 && !to_partial) return run_fwd(c, st);  // nothing to split
+  const int bn = splitkv_bn(D);
+  int ns = num_splits > 0 ? num_splits
+                          : fa_splitkv_default_splits(B, Sq, Sk, Hq, c.Hkv, D, num_sms(dev));
+  const long long tiles = std::max<long long>(1, ((long long)Sk + bn - 1) / bn);
+  if (ns > tiles) ns = (int)tiles;
+  const int split_keys = (int)(((tiles + ns - 1) / ns) * bn);
+  ns = (int)std::max<long long>(1, ((long long)Sk + split_keys - 1) / split_keys);
+  const long long rows = (long long)B * Sq * Hq;
+  const bool direct = to_partial && ns == 1;
+  if (!direct) {
+    const size_t need = fa_splitkv_workspace_bytes(B, Sq, Hq, D, ns);
+    if (workspace == nullptr || workspace_bytes < need)
+      return fail(FA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
+                  workspace_bytes);
+    if (!aligned16(workspace)) return fail(FA_ERR_INVALID, "workspace must be 16-byte aligned");
+  }
+  FwdParams p;
+  if ((s = fill_params(c, p, 1, bn, ns, split_keys)) != FA_OK) return s;
+  if (direct) {
+    p.o_part = static_cast<float *>(c.out);
+    p.lse_part = c.lse;
+  } else {
+    p.o_part = static_cast<float *>(workspace);
+    p.lse_part = p.o_part + (size_t)ns * rows * D;
+  }
+  const bool half = c.dt == FA_FP16;
+  if (D == 64)
+    s = launch_variant<Spl64>(p, dev, st, half, uses_mods(p));
+  else if (D == 128)
+    s = launch_variant<Spl128>(p, dev, st, half, uses_mods(p));
+  else
+    s = launch_variant<Spl256>(p, dev, st, half, uses_mods(p));
+  if (s != FA_OK || direct) return s;
+  return combine(D, half, to_partial, p.o_part, p.lse_part, ns, rows, c.out, c.lse, Hq, Sq, B,
+                 st);
+}
 
 }  // namespace
 
@@ -437,51 +514,43 @@ fa_status fa_fwd_splitkv_ex(const void *q, const void *k, const void *v, void *o
   Common c{q, k, v, out, lse, nullptr, nullptr, seqused_k, rel_bias, rel_extent, B, Sq, Sk,
            Hq, Hkv, D, 0, 0, 0, dt, causal, softmax_scale, false};
   apply_mods(c, mods);
-  fa_status s = validate(c);
-  if (s != FA_OK) return s;
-  if (num_splits < 0) return fail(FA_ERR_INVALID, "num_splits must be >= 0");
-  if ((long long)B * Sq == 0) return FA_OK;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return fail(FA_ERR_CUDA, "cudaGetDevice failed");
-  if (Sk == 0) return run_fwd(c, st);  // nothing to split
-  const int bn = splitkv_bn(D);
-  int ns = num_splits > 0 ? num_splits : fa_splitkv_default_splits(B, Sq, Sk, Hq, Hkv, D, num_sms(dev));
-  long long tiles = ((long long)Sk + bn - 1) / bn;
-  if (ns > tiles) ns = (int)tiles;
-  const int split_keys = (int)(((tiles + ns - 1) / ns) * bn);
-  ns = (int)(((long long)Sk + split_keys - 1) / split_keys);
-  const size_t need = fa_splitkv_workspace_bytes(B, Sq, Hq, D, ns);
-  if (workspace == nullptr || workspace_bytes < need)
-    return fail(FA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
-  if (!aligned16(workspace)) return fail(FA_ERR_INVALID, "workspace must be 16-byte aligned");
-  FwdParams p;
-  if ((s = fill_params(c, p, 1, bn, ns, split_keys)) != FA_OK) return s;
+  return run_splitkv(c, num_splits, workspace, workspace_bytes, false,
+                     static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_fwd_shard_partial(const void *q, const void *k, const void *v, float *o_part,
+                               float *lse_part, int B, int Sq, int Sk, int Hq, int Hkv, int D,
+                               fa_dtype dt, int causal, float softmax_scale,
+                               const int *seqused_k, const int *k_after, const void *rel_bias,
+                               int rel_extent, const fa_mods *mods, int num_splits,
+                               void *workspace, size_t workspace_bytes, void *stream) {
+  g_msg[0] = 0;
+  if (lse_part == nullptr && (long long)B * Sq > 0)
+    return fail(FA_ERR_INVALID, "lse_part must not be NULL");
+  Common c{q, k, v, o_part, lse_part, nullptr, nullptr, seqused_k, rel_bias, rel_extent, B,
+           Sq, Sk, Hq, Hkv, D, 0, 0, 0, dt, causal, softmax_scale, false};
+  apply_mods(c, mods);
+  c.k_after = k_after;
+  return run_splitkv(c, num_splits, workspace, workspace_bytes, true,
+                     static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_combine_partials(const float *o_parts, const float *lse_parts, int n_parts, int B,
+                              int Sq, int Hq, int D, fa_dtype dt, void *out, float *lse,
+                              void *stream) {
+  g_msg[0] = 0;
+  if (dt != FA_BF16 && dt != FA_FP16) return fail(FA_ERR_INVALID, "dtype must be bf16 or fp16");
+  if (B < 0 || Sq < 0 || Hq <= 0) return fail(FA_ERR_INVALID, "B, Sq must be >= 0 and Hq > 0");
+  if (D != 64 && D != 128 && D != 256)
+    return fail(FA_ERR_UNSUPPORTED, "head_dim %d not served (64, 128 or 256)", D);
+  if (n_parts < 1) return fail(FA_ERR_INVALID, "n_parts must be >= 1");
   const long long rows = (long long)B * Sq * Hq;
-  p.o_part = static_cast<float *>(workspace);
-  p.lse_part = p.o_part + (size_t)ns * rows * D;
-  const bool half = dt == FA_FP16;
-  if (D == 64)
-    s = launch_variant<Spl64>(p, dev, st, half, uses_mods(p));
-  else if (D == 128)
-    s = launch_variant<Spl128>(p, dev, st, half, uses_mods(p));
-  else
-    s = launch_variant<Spl256>(p, dev, st, half, uses_mods(p));
-  if (s != FA_OK) return s;
-  if (D == 64)
-    return half ? launch_combine<64, true>(p.o_part, p.lse_part, ns, rows, out, lse, Hq, Sq,
-                                           B * Sq, 1, st)
-                : launch_combine<64, false>(p.o_part, p.lse_part, ns, rows, out, lse, Hq, Sq,
-                                            B * Sq, 1, st);
-  if (D == 128)
-    return half ? launch_combine<128, true>(p.o_part, p.lse_part, ns, rows, out, lse, Hq, Sq,
-                                            B * Sq, 1, st)
-                : launch_combine<128, false>(p.o_part, p.lse_part, ns, rows, out, lse, Hq, Sq,
-                                             B * Sq, 1, st);
-  return half ? launch_combine<256, true>(p.o_part, p.lse_part, ns, rows, out, lse, Hq, Sq,
-                                          B * Sq, 1, st)
-              : launch_combine<256, false>(p.o_part, p.lse_part, ns, rows, out, lse, Hq, Sq,
-                                           B * Sq, 1, st);
+  if (rows == 0) return FA_OK;
+  if ((long long)B * Sq > 0x7fffffffLL) return fail(FA_ERR_UNSUPPORTED, "too many tokens");
+  if (!o_parts || !lse_parts || !out) return fail(FA_ERR_INVALID, "o_parts, lse_parts and out must not be NULL");
+  if (!aligned16(o_parts) || !aligned16(out)) return fail(FA_ERR_INVALID, "o_parts/out must be 16-byte aligned");
+  return combine(D, dt == FA_FP16, false, o_parts, lse_parts, n_parts, rows, out, lse, Hq, Sq, B,
+                 static_cast<cudaStream_t>(stream));
 }
 
 fa_status fa_watchdog_selftest(unsigned long long timeout_ns, void *stream) {

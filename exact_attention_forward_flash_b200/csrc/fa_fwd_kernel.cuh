@@ -127,6 +127,9 @@ struct FwdParams {
   float *lse_part;               // split partial LSE [splits][tok*Hq]
   const int *cu_q, *cu_k;        // varlen offsets, nullptr when dense
   const int *seqused_k;          // nullptr or [B]
+  // nullptr or [B]: keys of the whole sequence that follow the ones this
+  // call holds (a key shard); they move every row's diagonal that far right
+  const int *k_after;
   const uint16_t *rel_bias;      // nullptr or [tok, Hq, R]
   int R;
   int B, Sq, Sk, Hq, Hkv, G, P, lgP, n_groups;
@@ -271,6 +274,7 @@ __device__ __forceinline__ bool decode_unit(const FwdParams &p, const Sched &sch
   for (int t = 0; t < NQ; ++t)
     if ((U.row0 + t * kBM) / p.P < U.q_len) U.active |= 1u << t;
   U.delta = U.k_len - U.q_len;
+  if (p.k_after != nullptr) U.delta += min(max(__ldg(p.k_after + U.b), 0), 1 << 30);
   long long lo = (long long)U.split * p.split_keys;
   long long hi = min((long long)U.k_len, lo + p.split_keys);
   // keys no row of the unit admits are not visited: the window (causal is
@@ -1234,9 +1238,11 @@ __global__ void __launch_bounds__(32) fa_watchdog_selftest_kernel(unsigned long 
 }
 
 // ---------------------------------------------------------------------------
-// split-KV merge: one warp per packed (token, head) row
+// split-KV merge: one warp per packed (token, head) row.  F32OUT writes the
+// merged O in fp32 and its LSE at the row's own index, i.e. one more partial
+// in the layout the splits use (a key shard's partial, merged again later).
 // ---------------------------------------------------------------------------
-template <int D, bool HALF>
+template <int D, bool HALF, bool F32OUT = false>
 __global__ void __launch_bounds__(256) fa_combine_kernel(const float *__restrict__ o_part,
                                                          const float *__restrict__ lse_part,
                                                          int ns, long long rows, void *out,
@@ -1302,6 +1308,20 @@ __global__ void __launch_bounds__(256) fa_combine_kernel(const float *__restrict
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[e] += w[u] * x[u][e];
     }
+  }
+  if constexpr (F32OUT) {
+    float *dst = reinterpret_cast<float *>(out) + r * D + lane * E;
+    if constexpr (E % 4 == 0) {
+#pragma unroll
+      for (int e = 0; e < E; e += 4)
+        *reinterpret_cast<float4 *>(dst + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; e += 2)
+        *reinterpret_cast<float2 *>(dst + e) = make_float2(acc[e], acc[e + 1]);
+    }
+    if (lane == 0) lse[r] = Lse;
+    return;
   }
   uint16_t *dst = reinterpret_cast<uint16_t *>(out) + r * D + lane * E;
   if constexpr (E % 4 == 0) {

@@ -211,6 +211,47 @@ fa_status fa_fwd_splitkv_ex(const void *q, const void *k, const void *v,
                             void *stream);
 
 /*
+ * Context-parallel attention over key shards ("FlashAttention-4 backend for
+ * Blackwell #1235": the returned LSE lets a split over keys be merged outside
+ * the kernel; "mgoin/tml-fa4": the split-KV combine).  Each GPU holds one
+ * contiguous shard of every sequence's keys and values; the exact result is
+ * the LSE-weighted merge of the shards' normalised partials.
+ *
+ * fa_fwd_shard_partial: the partial of the shard held in k/v [B, Sk, Hkv, D]
+ * (dense layout; q [B, Sq, Hq, D] holds all query rows).  Masks and bias use
+ * the rows' distances in the WHOLE sequence: k_after (device int32 [B], or
+ * NULL for all zero) gives, per sequence, how many of its keys follow this
+ * shard, so d = i + (k_len + k_after[b] - q_len) - j with j the key's index
+ * within the shard and k_len = Sk (or seqused_k[b]).  Values are clamped to
+ * [0, 2^30].  rel_bias, causal and mods are those of the whole problem.
+ *   o_part   : device float [B*Sq*Hq][D], packed (token, head) rows, the
+ *              normalised partial O of this shard (0 for a row with no key);
+ *   lse_part : device float [B*Sq*Hq], its natural-log LSE (-inf, no key).
+ *   num_splits, workspace, workspace_bytes: as fa_fwd_splitkv (the shard's
+ *              keys are split again inside the GPU and merged into the one
+ *              partial); with one split the workspace may be NULL.
+ * A shard with Sk = 0 writes O = 0 and LSE = -inf for every row.
+ *
+ * fa_combine_partials: merges n_parts partials stacked as o_parts
+ * [n_parts][B*Sq*Hq][D] and lse_parts [n_parts][B*Sq*Hq] (the shards in any
+ * order) into out [B, Sq, Hq, D] of type dt and lse [B, Hq, Sq] (may be
+ * NULL).  A row whose partials are all -inf gets O = 0 and LSE = -inf.
+ * o_parts and out must be 16-byte aligned.
+ */
+fa_status fa_fwd_shard_partial(const void *q, const void *k, const void *v,
+                               float *o_part, float *lse_part, int B, int Sq,
+                               int Sk, int Hq, int Hkv, int D, fa_dtype dt,
+                               int causal, float softmax_scale,
+                               const int *seqused_k, const int *k_after,
+                               const void *rel_bias, int rel_extent,
+                               const fa_mods *mods, int num_splits,
+                               void *workspace, size_t workspace_bytes,
+                               void *stream);
+fa_status fa_combine_partials(const float *o_parts, const float *lse_parts,
+                              int n_parts, int B, int Sq, int Hq, int D,
+                              fa_dtype dt, void *out, float *lse, void *stream);
+
+/*
  * Device-side watchdog.  Every wait inside the kernels is bounded; a kernel
  * that gives up records a code in a device word and returns without
  * trapping.  This call synchronises the current device, copies that word to

@@ -123,3 +123,21 @@ def test_watchdog_selftest_validates_its_limit(lib):
     # out of [1 ms, 1 s]: rejected before anything is enqueued
     assert lib.fa_watchdog_selftest(10, None) == FA_ERR_INVALID
     assert lib.fa_watchdog_selftest(5_000_000_000, None) == FA_ERR_INVALID
+
+
+def test_shard_partial_and_combine_validation(lib):
+    # shard partial: the same argument checks as the split-KV entry point
+    sp = lib.fa_fwd_shard_partial
+    args = lambda D=128, lse=A, ns=1: (A, A, A, A, lse, 1, 1, 16, 4, 2, D, 0, 0, 0.0,  # noqa: E731
+                                       None, None, None, 0, None, ns, None, 0, None)
+    assert sp(*args(D=96)) == FA_ERR_UNSUPPORTED
+    assert sp(*args(lse=None)) == FA_ERR_INVALID
+    assert sp(*args(ns=-1)) == FA_ERR_INVALID
+    # combine: part count, head dim, dtype and alignment are checked first
+    cp = lib.fa_combine_partials
+    assert cp(A, A, 0, 1, 1, 4, 128, 0, A, A, None) == FA_ERR_INVALID
+    assert cp(A, A, 2, 1, 1, 4, 96, 0, A, A, None) == FA_ERR_UNSUPPORTED
+    assert cp(A, A, 2, 1, 1, 4, 128, 7, A, A, None) == FA_ERR_INVALID
+    assert cp(MIS, A, 2, 1, 1, 4, 128, 0, A, A, None) == FA_ERR_INVALID
+    assert cp(A, A, 2, 1, 1, 4, 128, 0, None, A, None) == FA_ERR_INVALID
+    assert cp(A, A, 2, 0, 1, 4, 128, 0, A, A, None) == FA_OK  # no rows: nothing to do
