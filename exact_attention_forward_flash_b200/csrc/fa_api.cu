@@ -100,11 +100,16 @@ fa_status encode_map(CUtensorMap *tm, const void *base, int D, int H, long long 
   if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)tokens};
   cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)box_h, (cuuint32_t)box_t};
+  // head dims that are a multiple of 64: 64-column boxes, 128-byte swizzle;
+  // narrow ones: 16-column boxes, 32-byte swizzle (the columns past D of the
+  // last box read as zero)
+  const bool narrow = D % 64 != 0;
+  cuuint32_t box[3] = {narrow ? 16u : 64u, (cuuint32_t)box_h, (cuuint32_t)box_t};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = fn(tm, half ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                   const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  narrow ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return FA_OK;
@@ -129,9 +134,15 @@ int num_sms(int dev) {
 
 // kernel variants
 // kernel configurations by (16-bit format: bf16 / fp16, modifiers off / on)
+template <bool H, bool M> using Fwd16 = FwdCfg<16, 128, 2, 1, 3, 0, H, false, M>;
+template <bool H, bool M> using Fwd48 = FwdCfg<48, 128, 2, 1, 3, 0, H, false, M>;
+template <bool H, bool M> using Fwd80 = FwdCfg<80, 128, 2, 1, 3, 0, H, false, M>;
 template <bool H, bool M> using Fwd64 = FwdCfg<64, 128, 2, 1, 3, 0, H, false, M>;
 template <bool H, bool M> using Fwd128 = FwdCfg<128, 128, 2, 1, 3, 0, H, false, M>;
 template <bool H, bool M> using Fwd256 = FwdCfg<256, 64, 1, 2, 3, 2, H, false, M>;
+template <bool H, bool M> using Spl16 = FwdCfg<16, 128, 1, 2, 3, 3, H, true, M>;
+template <bool H, bool M> using Spl48 = FwdCfg<48, 128, 1, 2, 3, 3, H, true, M>;
+template <bool H, bool M> using Spl80 = FwdCfg<80, 128, 1, 2, 3, 3, H, true, M>;
 template <bool H, bool M> using Spl64 = FwdCfg<64, 128, 1, 2, 3, 3, H, true, M>;
 template <bool H, bool M> using Spl128 = FwdCfg<128, 128, 1, 2, 3, 3, H, true, M>;
 template <bool H, bool M> using Spl256 = FwdCfg<256, 64, 1, 2, 2, 2, H, true, M>;
@@ -196,13 +207,19 @@ void apply_mods(Common &c, const fa_mods *m) {
   c.softcap = m->softcap;
 }
 
+// Head dims with a kernel: 64, 128, 256, and the narrow ones served by
+// 16-column-chunk kernels of width 16, 48 or 80 (D = 72 padded to 80).
+bool head_dim_served(int D) {
+  return D == 16 || D == 48 || D == 64 || D == 72 || D == 80 || D == 128 || D == 256;
+}
+
 fa_status validate(const Common &c) {
   if (c.dt != FA_BF16 && c.dt != FA_FP16) return fail(FA_ERR_INVALID, "dtype must be bf16 or fp16");
   if (c.B < 0 || c.Hq <= 0 || c.Hkv <= 0 || c.D <= 0)
     return fail(FA_ERR_INVALID, "B must be >= 0 and Hq, Hkv, D > 0");
   if (c.Hq % c.Hkv != 0) return fail(FA_ERR_INVALID, "Hq (%d) must be a multiple of Hkv (%d)", c.Hq, c.Hkv);
-  if (c.D != 64 && c.D != 128 && c.D != 256)
-    return fail(FA_ERR_UNSUPPORTED, "head_dim %d not served (64, 128 or 256)", c.D);
+  if (!head_dim_served(c.D))
+    return fail(FA_ERR_UNSUPPORTED, "head_dim %d not served (16, 48, 64, 72, 80, 128 or 256)", c.D);
   if (!c.varlen && (c.Sq < 0 || c.Sk < 0)) return fail(FA_ERR_INVALID, "Sq, Sk must be >= 0");
   if (c.varlen && (c.total_q < 0 || c.total_k < 0 || c.max_q < 0))
     return fail(FA_ERR_INVALID, "total_q, total_k, max_seqlen_q must be >= 0");
@@ -263,6 +280,7 @@ fa_status fill_params(const Common &c, FwdParams &p, int nq, int bn, int num_spl
   p.k_after = c.k_after;
   p.rel_bias = static_cast<const uint16_t *>(c.rel_bias);
   p.R = c.rel_bias ? c.R : 0;
+  p.d_out = c.D;
   p.B = c.B;
   p.Sq = c.Sq;
   p.Sk = c.Sk;
@@ -313,6 +331,9 @@ fa_status run_fwd(const Common &c, cudaStream_t st) {
   if (p.num_units == 0) return FA_OK;
   const bool half = c.dt == FA_FP16;
   const bool mods = uses_mods(p);
+  if (c.D == 16) return launch_variant<Fwd16>(p, dev, st, half, mods);
+  if (c.D == 48) return launch_variant<Fwd48>(p, dev, st, half, mods);
+  if (c.D == 72 || c.D == 80) return launch_variant<Fwd80>(p, dev, st, half, mods);
   if (c.D == 64) return launch_variant<Fwd64>(p, dev, st, half, mods);
   if (c.D == 128) return launch_variant<Fwd128>(p, dev, st, half, mods);
   return launch_variant<Fwd256>(p, dev, st, half, mods);
@@ -347,6 +368,23 @@ fa_status combine(int D, bool half, bool f32out, const float *o_part, const floa
                                                 tq, 1, st)                                   \
               : launch_combine<DD, false, false>(o_part, lse_part, ns, rows, out, lse, Hq,  \
                                                  Sq, tq, 1, st);
+  if (D % 64 != 0) {
+    const int warps = 8;
+    const long long blocks = (rows + warps - 1) / warps;
+    if (blocks > 0x7fffffffLL) return fail(FA_ERR_UNSUPPORTED, "too many rows");
+    if (f32out)
+      fa_combine_narrow_kernel<false, true><<<(unsigned)blocks, warps * 32, 0, st>>>(
+          o_part, lse_part, ns, rows, D, out, lse, Hq, Sq);
+    else if (half)
+      fa_combine_narrow_kernel<true, false><<<(unsigned)blocks, warps * 32, 0, st>>>(
+          o_part, lse_part, ns, rows, D, out, lse, Hq, Sq);
+    else
+      fa_combine_narrow_kernel<false, false><<<(unsigned)blocks, warps * 32, 0, st>>>(
+          o_part, lse_part, ns, rows, D, out, lse, Hq, Sq);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(FA_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
+    return FA_OK;
+  }
   if (D == 64) { FA_COMBINE(64) }
   if (D == 128) { FA_COMBINE(128) }
   FA_COMBINE(256)
@@ -397,7 +435,13 @@ fa_status run_splitkv(const Common &c, int num_splits, void *workspace, size_t w
     p.lse_part = p.o_part + (size_t)ns * rows * D;
   }
   const bool half = c.dt == FA_FP16;
-  if (D == 64)
+  if (D == 16)
+    s = launch_variant<Spl16>(p, dev, st, half, uses_mods(p));
+  else if (D == 48)
+    s = launch_variant<Spl48>(p, dev, st, half, uses_mods(p));
+  else if (D == 72 || D == 80)
+    s = launch_variant<Spl80>(p, dev, st, half, uses_mods(p));
+  else if (D == 64)
     s = launch_variant<Spl64>(p, dev, st, half, uses_mods(p));
   else if (D == 128)
     s = launch_variant<Spl128>(p, dev, st, half, uses_mods(p));
@@ -541,8 +585,8 @@ fa_status fa_combine_partials(const float *o_parts, const float *lse_parts, int 
   g_msg[0] = 0;
   if (dt != FA_BF16 && dt != FA_FP16) return fail(FA_ERR_INVALID, "dtype must be bf16 or fp16");
   if (B < 0 || Sq < 0 || Hq <= 0) return fail(FA_ERR_INVALID, "B, Sq must be >= 0 and Hq > 0");
-  if (D != 64 && D != 128 && D != 256)
-    return fail(FA_ERR_UNSUPPORTED, "head_dim %d not served (64, 128 or 256)", D);
+  if (!head_dim_served(D))
+    return fail(FA_ERR_UNSUPPORTED, "head_dim %d not served (16, 48, 64, 72, 80, 128 or 256)", D);
   if (n_parts < 1) return fail(FA_ERR_INVALID, "n_parts must be >= 1");
   const long long rows = (long long)B * Sq * Hq;
   if (rows == 0) return FA_OK;

@@ -132,6 +132,7 @@ struct FwdParams {
   const int *k_after;
   const uint16_t *rel_bias;      // nullptr or [tok, Hq, R]
   int R;
+  int d_out;         // head dim of the tensors (the kernel's D, or less with zero padding)
   int B, Sq, Sk, Hq, Hkv, G, P, lgP, n_groups;
   int total_q;
   int n_mblk;        // CTA tiles per (batch, head group, split)
@@ -302,16 +303,17 @@ __device__ __forceinline__ int unit_of(int k) {
   return k * G + ((k & 1) ? (G - 1 - c) : c);
 }
 
-// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout: start
-// address, leading and stride byte offsets in 16-byte units, version 1,
-// layout type 2 = SWIZZLE_128B).
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+// Shared-memory matrix descriptor (sm_100 layout: start address, leading and
+// stride byte offsets in 16-byte units, version 1, layout type in the top
+// bits: 2 = SWIZZLE_128B, 6 = SWIZZLE_32B).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout) {
   uint64_t d = 0;
   d |= (uint64_t)((addr & 0x3FFFFu) >> 4);
   d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
   d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
   d |= 1ull << 46;
-  d |= 2ull << 61;
+  d |= (uint64_t)(layout & 7u) << 61;
   return d;
 }
 
@@ -333,11 +335,21 @@ struct FwdCfg {
   // score/mask modifiers beyond causal (left window bound, soft-cap): a
   // separate kernel, so that the plain one carries none of their cost
   static constexpr bool MODS = MODS_;
-  static constexpr int kChunks = D / 64;          // 128-byte column chunks of a row
+  // Row chunks: 64 columns with a 128-byte swizzle when D is a multiple of
+  // 64; otherwise (narrow head dims, D a multiple of 16 holding a head dim
+  // padded up by zero-filled loads) 16 columns with a 32-byte swizzle.
+  static constexpr bool kNarrow = D % 64 != 0;
+  static constexpr int kCE = kNarrow ? 16 : 64;           // columns of a chunk
+  static constexpr int kCB = 2 * kCE;                     // bytes of a chunk row
+  static constexpr int kChunks = D / kCE;
   static constexpr int kQTile = kBM * D * 2;      // bytes
   static constexpr int kKVTile = BN * D * 2;
-  static constexpr int kQChunk = kBM * 128;       // bytes of one 64-column chunk
-  static constexpr int kKVChunk = BN * 128;
+  static constexpr int kQChunk = kBM * kCB;       // bytes of one chunk
+  static constexpr int kKVChunk = BN * kCB;
+  static constexpr uint32_t kSBO = 8 * kCB;       // stride of 8-row groups
+  static constexpr uint32_t kLayout = kNarrow ? 6u : 2u;
+  static constexpr int kKPerChunk = kCE / 16;     // 16-column MMA steps per chunk
+  static constexpr int kOStride = (D + 31) / 32 * 32;  // tensor-memory columns of one O
   static constexpr int kQOff = 0;
   // K/V stages: separate rings of KST and VST slots, or (VST == 0) one ring of
   // KST slots that the K and V tiles take in turn -- K(n), V(n), K(n+1), ...
@@ -382,9 +394,10 @@ struct FwdCfg {
   static_assert(!kSplitRegs || 128 * kRegsCtl + 256 * kRegsSoftmax <= 384 * 168, "register split");
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kOColBase = NQ * NS * BN;
-  static_assert(kOColBase + NQ * D <= 512, "tensor memory budget");
+  static_assert(kOColBase + NQ * kOStride <= 512, "tensor memory budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(D % 64 == 0 && BN % 32 == 0 && (BN == 64 || BN == 128), "tile shape");
+  static_assert((D % 64 == 0 || (D % 16 == 0 && D < 128)) && BN % 32 == 0 &&
+                    (BN == 64 || BN == 128), "tile shape");
   // slot and phase parity of the K tile k / V tile v (counted over the CTA's
   // whole sequence of KV tiles), and the barriers of V slots
   __host__ __device__ static constexpr uint32_t k_slot(uint32_t k) {
@@ -400,7 +413,7 @@ struct FwdCfg {
     return kKVRing ? ((2u * v + 1u) / KST) & 1u : (v / VST) & 1u;
   }
   __host__ __device__ static constexpr int s_col(int t, int b) { return (t * NS + b) * BN; }
-  __host__ __device__ static constexpr int o_col(int t) { return kOColBase + t * D; }
+  __host__ __device__ static constexpr int o_col(int t) { return kOColBase + t * kOStride; }
 };
 
 // ---------------------------------------------------------------------------
@@ -507,7 +520,7 @@ __device__ __forceinline__ void role_producer(const FwdParams &p, uint32_t sb) {
         mbar_arrive_expect_tx(bar(C::bQFull + t), C::kQTile);
 #pragma unroll
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(sb + C::kQOff + t * C::kQTile + c * C::kQChunk, &p.tm_q, c * 64, U.hq0, tok,
+          tma_load_3d(sb + C::kQOff + t * C::kQTile + c * C::kQChunk, &p.tm_q, c * C::kCE, U.hq0, tok,
                       bar(C::bQFull + t));
       }
       __syncwarp();
@@ -524,7 +537,7 @@ __device__ __forceinline__ void role_producer(const FwdParams &p, uint32_t sb) {
           mbar_arrive_expect_tx(bar(C::bKFull + s), C::kKVTile);
 #pragma unroll
           for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(sb + C::kKOff + s * C::kKVTile + c * C::kKVChunk, &p.tm_k, c * 64, U.hk,
+            tma_load_3d(sb + C::kKOff + s * C::kKVTile + c * C::kKVChunk, &p.tm_k, c * C::kCE, U.hk,
                         tok, bar(C::bKFull + s));
         }
         __syncwarp();
@@ -539,7 +552,7 @@ __device__ __forceinline__ void role_producer(const FwdParams &p, uint32_t sb) {
           mbar_arrive_expect_tx(bar(C::bVFull + s), C::kKVTile);
 #pragma unroll
           for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(sb + C::kVOff + s * C::kKVTile + c * C::kKVChunk, &p.tm_v, c * 64, U.hk,
+            tma_load_3d(sb + C::kVOff + s * C::kKVTile + c * C::kKVChunk, &p.tm_v, c * C::kCE, U.hk,
                         tok, bar(C::bVFull + s));
         }
         __syncwarp();
@@ -588,9 +601,12 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
     const uint32_t d_tmem = tmem + C::s_col(t, g % C::NS);
 #pragma unroll
     for (int kk = 0; kk < C::D / 16; ++kk) {
-      const uint32_t off = (kk % 4) * 32;  // 16 elements = 32 bytes inside the swizzle atom
-      const uint64_t a = smem_desc_sw128(qa + (kk / 4) * C::kQChunk + off, 16, 1024);
-      const uint64_t b = smem_desc_sw128(ka + (kk / 4) * C::kKVChunk + off, 16, 1024);
+      // 16 elements = 32 bytes inside the swizzle atom
+      const uint32_t off = (kk % C::kKPerChunk) * 32;
+      const uint64_t a = smem_desc(qa + (kk / C::kKPerChunk) * C::kQChunk + off, 16, C::kSBO,
+                                   C::kLayout);
+      const uint64_t b = smem_desc(ka + (kk / C::kKPerChunk) * C::kKVChunk + off, 16, C::kSBO,
+                                   C::kLayout);
       tc_mma_ss_elect(d_tmem, a, b, idesc_s, kk > 0 ? 1u : 0u);
     }
     tc_commit_elect(bar(C::bSFull + t * C::NS + g % C::NS));
@@ -603,8 +619,8 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
     const uint32_t d_tmem = tmem + C::o_col(t);
 #pragma unroll
     for (int kk = 0; kk < C::BN / 16; ++kk) {
-      // 16 keys = two 8-row groups (SBO 1024 B); 64-column chunks LBO apart
-      const uint64_t b = smem_desc_sw128(va + kk * 16 * 128, C::kKVChunk, 1024);
+      // 16 keys = two 8-row groups (SBO apart); column chunks LBO apart
+      const uint64_t b = smem_desc(va + kk * 16 * C::kCB, C::kKVChunk, C::kSBO, C::kLayout);
       tc_mma_ts_elect(d_tmem, p_tmem + kk * 8, b, idesc_pv, (first && kk == 0) ? 0u : 1u);
     }
     tc_commit_elect(bar(C::bOFull + t * C::NS + g % C::NS));
@@ -614,13 +630,15 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
   constexpr uint32_t idesc_s64 = instr_desc<C::HALF>(kBM, 64, false, false);
   auto issue_s_half = [&](int t, uint32_t g, uint32_t kstage, int hi) {
     const uint32_t qa = sb + C::kQOff + t * C::kQTile;
-    const uint32_t ka = sb + C::kKOff + kstage * C::kKVTile + hi * 64 * 128;
+    const uint32_t ka = sb + C::kKOff + kstage * C::kKVTile + hi * 64 * C::kCB;
     const uint32_t d_tmem = tmem + C::s_col(t, g % C::NS) + hi * 64;
 #pragma unroll
     for (int kk = 0; kk < C::D / 16; ++kk) {
-      const uint32_t off = (kk % 4) * 32;
-      const uint64_t a = smem_desc_sw128(qa + (kk / 4) * C::kQChunk + off, 16, 1024);
-      const uint64_t b = smem_desc_sw128(ka + (kk / 4) * C::kKVChunk + off, 16, 1024);
+      const uint32_t off = (kk % C::kKPerChunk) * 32;
+      const uint64_t a = smem_desc(qa + (kk / C::kKPerChunk) * C::kQChunk + off, 16, C::kSBO,
+                                   C::kLayout);
+      const uint64_t b = smem_desc(ka + (kk / C::kKPerChunk) * C::kKVChunk + off, 16, C::kSBO,
+                                   C::kLayout);
       tc_mma_ss_elect(d_tmem, a, b, idesc_s64, kk > 0 ? 1u : 0u);
     }
   };
@@ -632,7 +650,7 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
 #pragma unroll
     for (int k4 = 0; k4 < 4; ++k4) {
       const int kk = 4 * hi + k4;
-      const uint64_t b = smem_desc_sw128(va + kk * 16 * 128, C::kKVChunk, 1024);
+      const uint64_t b = smem_desc(va + kk * 16 * C::kCB, C::kKVChunk, C::kSBO, C::kLayout);
       tc_mma_ts_elect(d_tmem, p_tmem + kk * 8, b, idesc_pv, (first && kk == 0) ? 0u : 1u);
     }
   };
@@ -840,6 +858,9 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
                                              int t) {
   auto bar = [&](int i) { return sb + C::kBarOff + 8u * i; };
   constexpr int BN = C::BN, D = C::D, NS = C::NS;
+  // row pitch of the output: the tensors' head dim (narrow dims are padded
+  // in the kernel; their padding columns are never stored)
+  const int dO = C::kNarrow ? p.d_out : D;
   const int tid = static_cast<int>(threadIdx.x) - 128 * (t + 1);  // tile row == TMEM lane
   const int lane = tid & 31;
   const uint32_t lane_addr = static_cast<uint32_t>(tid & ~31) << 16;
@@ -868,10 +889,10 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
     float *lse_ptr;
     if constexpr (C::PARTIAL) {
       const size_t prow = (size_t)U.split * p.total_q * p.Hq + orow;
-      out_row = p.o_part + prow * D;
+      out_row = p.o_part + prow * dO;
       lse_ptr = p.lse_part + prow;
     } else {
-      out_row = reinterpret_cast<uint16_t *>(p.out) + orow * D;
+      out_row = reinterpret_cast<uint16_t *>(p.out) + orow * dO;
       lse_ptr = p.lse == nullptr ? nullptr
                 : p.lse + (p.lse_dense ? ((size_t)U.b * p.Hq + h) * p.Sq + i
                                        : (size_t)h * p.total_q + U.q_start + i);
@@ -920,7 +941,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
           }
           const uint32_t o_addr = tmem + lane_addr + C::o_col(t);
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < C::kOStride / 32; ++c) {
             uint32_t o[32];
             tmem_ld32(o_addr + 32 * c, o);
             tmem_wait_ld();
@@ -1116,7 +1137,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
     }
     if (warp_on) {
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < C::kOStride / 32; ++c) {
         uint32_t r[32];
         if (nb > 0) {
           tmem_ld32(tmem + lane_addr + C::o_col(t) + 32 * c, r);
@@ -1130,6 +1151,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
             float *dst = reinterpret_cast<float *>(out_row) + 32 * c;
 #pragma unroll
             for (int e = 0; e < 32; e += 4) {
+              if (C::kNarrow && 32 * c + e >= dO) break;
               float4 w = make_float4(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l,
                                      __uint_as_float(r[e + 2]) * inv_l,
                                      __uint_as_float(r[e + 3]) * inv_l);
@@ -1139,6 +1161,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
             uint16_t *dst = reinterpret_cast<uint16_t *>(out_row) + 32 * c;
 #pragma unroll
             for (int e = 0; e < 32; e += 8) {
+              if (C::kNarrow && 32 * c + e >= dO) break;
               uint4 w;
               w.x = pack2<C::HALF>(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l);
               w.y = pack2<C::HALF>(__uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
@@ -1343,6 +1366,65 @@ __global__ void __launch_bounds__(256) fa_combine_kernel(const float *__restrict
     const long long li =
         lse_dense ? ((tok / Sq) * Hq + h) * (long long)Sq + tok % Sq : (long long)h * total_q + tok;
     lse[li] = Lse;
+  }
+}
+
+// The same merge for narrow head dims d (a multiple of 8, at most 128): lane
+// l handles the column pairs starting at 2l and 2l + 64.
+template <bool HALF, bool F32OUT>
+__global__ void __launch_bounds__(256) fa_combine_narrow_kernel(const float *__restrict__ o_part,
+                                                                const float *__restrict__ lse_part,
+                                                                int ns, long long rows, int d,
+                                                                void *out, float *lse, int Hq,
+                                                                int Sq) {
+  const long long r = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const float L2E = 1.4426950408889634f;
+  float m = -INFINITY;
+  for (int s = lane; s < ns; s += 32) m = fmaxf(m, lse_part[(long long)s * rows + r]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float z = 0.f;
+  if (m != -INFINITY)
+    for (int s = lane; s < ns; s += 32) z += ex2_approx((lse_part[(long long)s * rows + r] - m) * L2E);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  const float Lse = (m == -INFINITY) ? -INFINITY : m + lg2_approx(z) * 0.69314718055994531f;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const int c0 = 2 * lane, c1 = 2 * lane + 64;
+  if (m != -INFINITY) {
+    for (int s = 0; s < ns; ++s) {
+      const float ls = __ldg(lse_part + (long long)s * rows + r);
+      if (ls == -INFINITY) continue;
+      const float w = ex2_approx((ls - Lse) * L2E);
+      const float *src = o_part + ((long long)s * rows + r) * d;
+      if (c0 < d) {
+        const float2 v = __ldg(reinterpret_cast<const float2 *>(src + c0));
+        acc[0] += w * v.x;
+        acc[1] += w * v.y;
+      }
+      if (c1 < d) {
+        const float2 v = __ldg(reinterpret_cast<const float2 *>(src + c1));
+        acc[2] += w * v.x;
+        acc[3] += w * v.y;
+      }
+    }
+  }
+  if constexpr (F32OUT) {
+    float *dst = reinterpret_cast<float *>(out) + r * d;
+    if (c0 < d) *reinterpret_cast<float2 *>(dst + c0) = make_float2(acc[0], acc[1]);
+    if (c1 < d) *reinterpret_cast<float2 *>(dst + c1) = make_float2(acc[2], acc[3]);
+    if (lane == 0) lse[r] = Lse;
+  } else {
+    uint16_t *dst = reinterpret_cast<uint16_t *>(out) + r * d;
+    if (c0 < d) *reinterpret_cast<uint32_t *>(dst + c0) = pack2<HALF>(acc[0], acc[1]);
+    if (c1 < d) *reinterpret_cast<uint32_t *>(dst + c1) = pack2<HALF>(acc[2], acc[3]);
+    if (lane == 0 && lse != nullptr) {
+      const long long tok = r / Hq;
+      const int h = (int)(r % Hq);
+      lse[((tok / Sq) * Hq + h) * (long long)Sq + tok % Sq] = Lse;
+    }
   }
 }
 

@@ -33,8 +33,10 @@
  *     synchronises the stream: a call only enqueues work on `stream`
  *     (a cudaStream_t; NULL means the legacy default stream) and returns.
  *   - Element type `dt` applies to q, k, v, out and rel_bias alike.
- *   - head_dim D must be 64, 128 or 256; Hq must be a multiple of Hkv; query head
- *     h reads K/V head h / (Hq / Hkv).
+ *   - head_dim D must be 16, 48, 64, 72, 80, 128 or 256 ("FlashAttention-4
+ *     backend for Blackwell #1235" uses head dims 16 and 64,
+ *     "flashrt/fa4-cute-runtime" the D48/D72/D128 family and D256); Hq must
+ *     be a multiple of Hkv; query head h reads K/V head h / (Hq / Hkv).
  *   - q, k, v, out and rel_bias must be 16-byte aligned and contiguous in the
  *     documented layout.  cu_seqlens and seqused_k are device int32 arrays.
  *   - softmax_scale <= 0 selects 1 / sqrt(D).

@@ -77,7 +77,7 @@ def test_decode_shards_merge_to_the_full_result(world, ns):
     compare(out, lse, ro, rl, what=f"cp decode world={world} ns={ns}")
 
 
-@pytest.mark.parametrize("D", [64, 128, 256])
+@pytest.mark.parametrize("D", [16, 64, 72, 128, 256])
 def test_causal_bias_seqused_shards(D):
     # several query rows, causal bottom-right diagonal, 128-wide bias and
     # padded keys: every rule that reads a key's global position

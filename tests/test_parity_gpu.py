@@ -85,6 +85,13 @@ CASES = [
     (1, 70, 600, 4, 4, 256, True),
     (2, 300, 300, 4, 4, 64, True),     # D=64
     (1, 129, 390, 8, 2, 64, False),    # D=64, group of 4 packed
+    # narrow head dims (16-column chunks, 32-byte swizzle; 72 padded to 80)
+    (2, 300, 300, 4, 4, 16, True),
+    (1, 129, 390, 8, 1, 16, False),    # D=16, MQA group of 8 packed
+    (1, 257, 300, 6, 2, 48, True),     # D=48, group of 3: heads not packed
+    (1, 300, 300, 8, 8, 72, True),     # D=72 MHA
+    (2, 129, 390, 8, 2, 72, False),
+    (1, 200, 333, 4, 2, 80, True),
 ]
 
 
@@ -97,7 +104,7 @@ def test_dense_shapes(case):
     compare(out, lse, ro, rl, what=str(case))
 
 
-@pytest.mark.parametrize("D", [64, 128, 256])
+@pytest.mark.parametrize("D", [16, 48, 64, 72, 128, 256])
 def test_fp16_causal_gqa(D):
     p = fa_inputs.random_dense(7, 2, 260, 270, 8, 2, D, dtype=torch.float16, causal=True)
     out, lse = run_dense(p)
@@ -108,7 +115,7 @@ def test_fp16_causal_gqa(D):
 # ---------------------------------------------------------------------------
 # varlen with empty / one-token / multi-tile sequences, causal, GQA, bias
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("D", [64, 128, 256])
+@pytest.mark.parametrize("D", [16, 48, 64, 72, 128, 256])
 @pytest.mark.parametrize("causal", [False, True])
 def test_varlen_bias(D, causal):
     q_lens = [0, 1, 130, 257, 513, 64]
@@ -210,7 +217,7 @@ def test_dense_d64_sampled():
 # split-KV
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("ns", [0, 1, 3, 7])
-@pytest.mark.parametrize("D", [64, 128, 256])
+@pytest.mark.parametrize("D", [16, 64, 72, 128, 256])
 def test_splitkv_small(ns, D):
     p = fa_inputs.random_dense(21 + D, 3, 1, 1000, 8, 2, D)
     g = p.to(DEV)
@@ -351,6 +358,8 @@ WINDOW_CASES = [
     (1, 300, 300, 8, 1, 256, True, (63, -1)),     # D = 256
     (2, 400, 650, 4, 2, 64, False, (300, 10)),    # D = 64
     (1, 260, 100, 4, 4, 128, False, (0, 0)),      # diagonal key only; early rows see none
+    (1, 500, 500, 4, 1, 16, True, (100, -1)),     # D = 16
+    (1, 400, 600, 4, 2, 72, False, (200, 50)),    # D = 72
 ]
 
 
@@ -363,7 +372,7 @@ def test_window(case):
     compare(out, lse, ro, rl, what=f"window {case}")
 
 
-@pytest.mark.parametrize("D", [64, 128, 256])
+@pytest.mark.parametrize("D", [16, 64, 72, 128, 256])
 @pytest.mark.parametrize("causal", [False, True])
 def test_softcap(D, causal):
     # q sharpened so that the cap matters (scaled scores well beyond it)
