@@ -37,7 +37,7 @@ if ROOT not in sys.path:
 METRIC = "attention fwd TFLOP/s & % of BF16 tensor peak; split-KV decode HBM GB/s"
 MAIN = "varlen_gqa_bias"
 EXTRAS = ["dense_257", "video_dit_20480", "encoder_d256_seqused", "decode_splitkv", "dense_d64",
-          "local_window_softcap"]
+          "local_window_softcap", "tabpfn_d16", "vision_d72"]
 DESCR = {
     "dense_257": "dense non-causal MHA B=1 S=257 H=8 D=128 bf16",
     "varlen_gqa_bias": "varlen causal GQA 32/8 D=128, 4 seqs U[512,4096] (seeded), rel_bias R=256 bf16",
@@ -46,6 +46,8 @@ DESCR = {
     "decode_splitkv": "split-KV decode B=8 Sq=1 Sk=131072 Hq=32 Hkv=8 D=128 bf16",
     "dense_d64": "dense non-causal MHA B=4 S=4096 H=16 D=64 bf16",
     "local_window_softcap": "causal GQA 16/4 D=128 B=1 S=32768, window 4095 left, softcap 50 bf16",
+    "tabpfn_d16": "dense non-causal MHA B=1 S=30000 H=8 D=16 fp16",
+    "vision_d72": "dense non-causal MHA B=32 S=729 H=16 D=72 bf16",
 }
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
 
@@ -339,6 +341,61 @@ def time_e2e(p, p_cpu, splits: int, steps: int, dist_on: bool, world: int, unit:
             "pipeline": "2 buffer sets, copy-in / compute / copy-out streams"}
 
 
+def time_short_calls(dev, n_calls: int = 2000, per_graph: int = 100, replays: int = 20):
+    """Per-call cost of a short forward: the query block of a cached
+    prediction (B=1, Sq=128, Sk=1024, MQA 8/1, D=64, fp16), called many times.
+    Reports the wall time per call of eager calls through the public API,
+    issued back to back (host marshalling + launch), and the device time per
+    call when the same calls are replayed from one CUDA graph."""
+    import torch
+    import fa_inputs
+    import exact_attention_forward_flash_b200 as fa
+    p = fa_inputs.random_dense(900, 1, 128, 1024, 8, 1, 64, dtype=torch.float16).to(dev)
+    out = torch.empty_like(p.q)
+    lse = torch.empty((1, 8, 128), dtype=torch.float32, device=dev)
+
+    ns = fa.splitkv_default_splits(1, 128, 1024, 8, 1, 64,
+                                   torch.cuda.get_device_properties(dev).multi_processor_count)
+    ws = torch.empty(max(16, fa.splitkv_workspace_bytes(1, 128, 8, 64, ns)), dtype=torch.uint8,
+                     device=dev)
+
+    def plain():
+        fa.fa_fwd(p.q, p.k, p.v, softmax_scale=p.softmax_scale, out=out, lse=lse)
+
+    def split():
+        fa.fa_fwd_splitkv(p.q, p.k, p.v, num_splits=ns, softmax_scale=p.softmax_scale,
+                          out=out, lse=lse, workspace=ws)
+
+    def measure(call):
+        for _ in range(20):
+            call()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(n_calls):
+            call()
+        torch.cuda.synchronize()
+        eager_us = (time.perf_counter() - t0) / n_calls * 1e6
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(per_graph):
+                call()
+        graph.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(replays):
+            graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        graph_us = e0.elapsed_time(e1) * 1e3 / (replays * per_graph)
+        del graph
+        return {"eager_us_per_call": round(eager_us, 2), "graph_us_per_call": round(graph_us, 2),
+                "graph_tflops": round(p.flops() / (graph_us * 1e-6) / 1e12, 2)}
+
+    return {"shape": "dense B=1 Sq=128 Sk=1024 Hq=8 Hkv=1 D=64 fp16",
+            "fa_fwd": measure(plain), "fa_fwd_splitkv": dict(measure(split), num_splits=ns)}
+
+
 def max_over_ranks(x: float, dist_on: bool) -> float:
     """The maximum of a per-rank time over all ranks (NCCL on the GPU, or a
     CPU tensor when the process group runs on gloo)."""
@@ -503,6 +560,11 @@ def main():
             del q, r
             torch.cuda.empty_cache()
 
+    # ---- many short calls: per-call overhead, eager and from a CUDA graph
+    short = None
+    if not a.no_extras:
+        short = time_short_calls(dev)
+
     # ---- CPU oracle on this host (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and p_cpu is not None:
@@ -532,6 +594,7 @@ def main():
         "clocks": clocks,
         "kernel_source_sha256": kernel_source_hash(),
         "workloads": extras,
+        "short_calls": short,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

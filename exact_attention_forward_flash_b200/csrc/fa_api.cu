@@ -529,7 +529,12 @@ int fa_splitkv_default_splits(int B, int Sq, int Sk, int Hq, int Hkv, int D, int
   const int P = pack_factor(Hq / Hkv);
   const long long mblk = ((long long)Sq * P + kBM - 1) / kBM;
   const long long base = (long long)B * (Hq / P) * mblk;  // units without splitting
-  const long long max_by_len = std::max<long long>(1, ((long long)Sk + 8 * bn - 1) / (8 * bn));
+  // splits of at least 8 key tiles keep a decode streaming; a short call
+  // whose units cover under a quarter of the SMs trades that for latency and
+  // splits down to 2 tiles
+  const int min_tiles = base * 4 >= n_sms ? 8 : 2;
+  const long long max_by_len =
+      std::max<long long>(1, ((long long)Sk + min_tiles * bn - 1) / (min_tiles * bn));
   if (base >= 4LL * n_sms) return 1;
   // enough units for about 16 per SM, in whole waves where possible
   long long ns = (16LL * n_sms + base - 1) / base;

@@ -367,6 +367,16 @@ struct FwdCfg {
   // can be computed as soon as the softmax has read S(n).  Measured slower:
   // 128x64 MMAs issue at ~50 cycles for 32 of work.
   static constexpr bool kSplitS = false;
+  // Separate P buffer (64 tensor-memory columns per Q tile, where S, O and P
+  // fit: D <= 64): P(n) no longer overwrites S(n), so S(n+1) is computed as
+  // soon as the softmax has read S(n), while it works on tile n, instead of
+  // after P(n).V.  The softmax then waits for P(n-1).V before it stores P(n)
+  // or rescales O.  Measured 9-15% slower at D = 16 and 64: the two tiles'
+  // softmaxes then run at the same time on the same SMSPs instead of taking
+  // turns, and their exponential and FMA work per SMSP does not shrink.
+  static constexpr bool kSepPWanted = false;
+  static constexpr bool kSepP = kSepPWanted && kSplitPV && NQ == 2 && !kSplitS &&
+                                NQ * NS * BN + NQ * ((D + 31) / 32 * 32) + NQ * (BN / 2) <= 512;
   // barrier indices
   static constexpr int bQFull = 0, bQEmpty = NQ, bKFull = 2 * NQ, bKEmpty = bKFull + KST,
                        bVFull0 = bKEmpty + KST, bVEmpty0 = bVFull0 + VST, bSFull = bVEmpty0 + VST,
@@ -394,7 +404,8 @@ struct FwdCfg {
   static_assert(!kSplitRegs || 128 * kRegsCtl + 256 * kRegsSoftmax <= 384 * 168, "register split");
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kOColBase = NQ * NS * BN;
-  static_assert(kOColBase + NQ * kOStride <= 512, "tensor memory budget");
+  static constexpr int kPColBase = kOColBase + NQ * kOStride;
+  static_assert(kPColBase + (kSepP ? NQ * BN / 2 : 0) <= 512, "tensor memory budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert((D % 64 == 0 || (D % 16 == 0 && D < 128)) && BN % 32 == 0 &&
                     (BN == 64 || BN == 128), "tile shape");
@@ -414,6 +425,10 @@ struct FwdCfg {
   }
   __host__ __device__ static constexpr int s_col(int t, int b) { return (t * NS + b) * BN; }
   __host__ __device__ static constexpr int o_col(int t) { return kOColBase + t * kOStride; }
+  // columns of P_t(g): its own buffer, or the first half of S_t(g)'s
+  __host__ __device__ static constexpr int p_col(int t, int b) {
+    return kSepP ? kPColBase + t * (BN / 2) : s_col(t, b);
+  }
 };
 
 // ---------------------------------------------------------------------------
@@ -615,7 +630,7 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
   // O_t += P_t(g) V (P in the S buffer of g, as 16-bit pairs)
   auto issue_pv = [&](int t, uint32_t g, uint32_t vstage, bool first) {
     const uint32_t va = sb + C::kVOff + vstage * C::kKVTile;
-    const uint32_t p_tmem = tmem + C::s_col(t, g % C::NS);
+    const uint32_t p_tmem = tmem + C::p_col(t, g % C::NS);
     const uint32_t d_tmem = tmem + C::o_col(t);
 #pragma unroll
     for (int kk = 0; kk < C::BN / 16; ++kk) {
@@ -645,7 +660,7 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
   // split form: O_t += P_t[:, 64 hi .. 64 hi + 64) V[64 hi .. 64 hi + 64, :]
   auto issue_pv_half = [&](int t, uint32_t g, uint32_t vstage, bool first, int hi) {
     const uint32_t va = sb + C::kVOff + vstage * C::kKVTile;
-    const uint32_t p_tmem = tmem + C::s_col(t, g % C::NS);
+    const uint32_t p_tmem = tmem + C::p_col(t, g % C::NS);
     const uint32_t d_tmem = tmem + C::o_col(t);
 #pragma unroll
     for (int k4 = 0; k4 < 4; ++k4) {
@@ -702,6 +717,28 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
       }
       const uint32_t vn = vb + n;
       bool k_next_ready = false;  // K tile n+1 waited for (split form)
+      if constexpr (C::kSepP) {
+        // S_t(n+1) for every tile as soon as its softmax has read S_t(n)
+        if (n + 1 < nb) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + C::k_slot(kn)), C::k_par(kn),
+                                                 &g_fa_error, p.timeout_ns));
+          if (!ok) break;
+          k_next_ready = true;
+#pragma unroll
+          for (int t = 0; t < C::NQ; ++t) {
+            if (!(U.active >> t & 1u)) continue;
+            const uint32_t g = sbase[t] + n;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bSRead + t), g & 1u, &g_fa_error,
+                                                   p.timeout_ns));
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(t, g + 1, C::k_slot(kn));  // commits the S barrier itself
+            if (n + 1 == nb - 1) tc_commit_elect(bar(C::bQEmpty + t));
+          }
+          if (!ok) break;
+          tc_commit_elect(bar(C::bKEmpty + C::k_slot(kn)));
+        }
+      }
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bVFull + C::v_slot(vn)), C::v_par(vn), &g_fa_error,
                      p.timeout_ns));
       if (!ok) break;
@@ -743,7 +780,7 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
           issue_pv_half(t, g, C::v_slot(vn), n == 0, 1);
           tc_commit_elect(bar(C::bOFull + t));
           if (t == last_t) tc_commit_elect(bar(C::bVEmpty + C::v_slot(vn)));
-          if (more) {
+          if (more && !C::kSepP) {
             if (C::kSplitS) {
               issue_s_half(t, g + 1, C::k_slot(kn), 0);
               tc_commit_elect(bar(C::bSFull + t));
@@ -910,6 +947,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
       const bool bias_blk = __any_sync(0xffffffffu, has_bias && valid && base >= 0 &&
                                                         base - (BN - 1) < p.R);
       const uint32_t s_addr = tmem + lane_addr + C::s_col(t, buf);
+      const uint32_t p_addr = tmem + lane_addr + C::p_col(t, buf);
       const int lim_c = lim_rel - jrel;  // columns at or past lim_c are masked
       const int st_c = C::MODS ? st_rel - jrel : 0;  // and columns before st_c
       // no row of the warp has a masked column here: the FMA-pipe exponential
@@ -932,7 +970,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
         // the previous P.V must have completed (guaranteed by the score
         // barrier when S is single-buffered, waited for otherwise).
         auto rescale_o = [&](float f) -> bool {
-          if (NS == 2) {
+          if (NS == 2 || C::kSepP) {
             const uint32_t gp = g - 1;
             if (!__all_sync(0xffffffffu, mbar_wait(bar(C::bOFull + t * NS + gp % NS),
                                                    (gp / NS) & 1u, &g_fa_error, p.timeout_ns)))
@@ -951,6 +989,15 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
           }
           return true;
         };
+      // separate P buffer: P(g-1).V must be done before P(g) overwrites it
+      auto wait_prev_pv = [&]() -> bool {
+        const uint32_t gp = g - 1;
+        const bool w = __all_sync(0xffffffffu, mbar_wait(bar(C::bOFull + t * NS + gp % NS),
+                                                         (gp / NS) & 1u, &g_fa_error,
+                                                         p.timeout_ns));
+        tc_fence_after();
+        return w;
+      };
       // The two kinds of tile take disjoint paths (each with its own wait) so
       // that their register-resident arrays never meet at a join.
       if (bias_blk) {
@@ -988,7 +1035,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
               }
             }
             // every score read: the next tile's upper keys may land
-            if (C::kSplitS && hf == BN / 64 - 1) warp_arrive(C::bSRead + t);
+            if ((C::kSplitS || C::kSepP) && hf == BN / 64 - 1) warp_arrive(C::bSRead + t);
             if constexpr (C::MODS) {
               if (p.cap_a > 0.f) softcap_all<64>(x, p.cap_a, p.cap_b);
             }
@@ -1023,12 +1070,12 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
 #pragma unroll 1
                 for (int c = 0; c < hf; ++c) {
                   uint32_t o[32];
-                  tmem_ld32(s_addr + 32 * c, o);
+                  tmem_ld32(p_addr + 32 * c, o);
                   tmem_wait_ld();
 #pragma unroll
                   for (int e = 0; e < 32; ++e)
                     o[e] = pack2<C::HALF>(lo_f<C::HALF>(o[e]) * f, hi_f<C::HALF>(o[e]) * f);
-                  tmem_st32(s_addr + 32 * c, o);
+                  tmem_st32(p_addr + 32 * c, o);
                 }
               }
               tmem_wait_st();
@@ -1041,13 +1088,26 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
           else
             l += exp_pack<C::HALF, false, 0, 64>(x, sl2, mc, pk);
           // P half hf -> columns [32 hf, 32 hf + 32): only score columns
-          // already read are overwritten
-          tmem_st32(s_addr + 32 * hf, pk);
+          // already read are overwritten (or the separate P buffer's)
+          if (C::kSepP && hf == 0 && n > 0) {
+            ok = wait_prev_pv();
+            if (!ok) break;
+          }
+          tmem_st32(p_addr + 32 * hf, pk);
           }
           if (!ok) break;
           tmem_wait_st();
-        } else if (C::kSplitS) {
-          warp_arrive(C::bSRead + t);
+        } else {
+          if (C::kSplitS || C::kSepP) warp_arrive(C::bSRead + t);
+          // A warp without rows must not run ahead: with a separate P buffer
+          // S(g+1) is ready while the other warps still work on tile g, and
+          // its P arrivals for g+1 would complete their phase for g.  Its
+          // arrivals for tile g wait until P(g-1).V is done, i.e. until every
+          // warp has finished tile g-1.
+          if (C::kSepP && n > 0) {
+            ok = wait_prev_pv();
+            if (!ok) break;
+          }
         }
         // the bias path may rescale its first P half after storing it, so the
         // first-half signal waits for the whole tile
@@ -1068,7 +1128,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
             for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(r[e]);
           }
           tmem_wait_ld();
-          if (C::kSplitS) warp_arrive(C::bSRead + t);
+          if (C::kSplitS || C::kSepP) warp_arrive(C::bSRead + t);
           if constexpr (C::MODS) {
             if (p.cap_a > 0.f) softcap_all<BN>(s, p.cap_a, p.cap_b);
           }
@@ -1100,7 +1160,11 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
               l += exp_pack<C::HALF, true, 0, 64>(s, sl2, mc, pk);
             else
               l += exp_pack<C::HALF, false, 0, 64>(s, sl2, mc, pk);
-            tmem_st32(s_addr, pk);
+            if (C::kSepP && n > 0) {
+              ok = wait_prev_pv();
+              if (!ok) break;
+            }
+            tmem_st32(p_addr, pk);
             if (C::kSplitPV) {
               tmem_wait_st();
               warp_arrive(C::bPHalf + t);
@@ -1112,12 +1176,16 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
               l += exp_pack<C::HALF, true, 64, 64>(s, sl2, mc, pk);
             else
               l += exp_pack<C::HALF, false, 64, 64>(s, sl2, mc, pk);
-            tmem_st32(s_addr + 32, pk);
+            tmem_st32(p_addr + 32, pk);
           }
           tmem_wait_st();
           warp_arrive(C::bPFull + t * NS + buf);
         } else {
-          if (C::kSplitS) warp_arrive(C::bSRead + t);
+          if (C::kSplitS || C::kSepP) warp_arrive(C::bSRead + t);
+          if (C::kSepP && n > 0) {  // no running ahead (see the bias path)
+            ok = wait_prev_pv();
+            if (!ok) break;
+          }
           if (C::kSplitPV) warp_arrive(C::bPHalf + t);
           warp_arrive(C::bPFull + t * NS + buf);
         }

@@ -24,6 +24,13 @@ Workloads (shapes from the pages' validation tables and API contracts):
 * ``local_window_softcap``: causal GQA 16/4, D=128, B=1, S=32768 with a
   sliding window of 4095 keys to the left and scores soft-capped at 50 (the
   pages' "mask/score modifiers", at local-attention sizes).
+* ``tabpfn_d16``: dense non-causal MHA, fp16, B=1, S=30000, H=8, D=16: the
+  head-dim-16 attention stages of "FlashAttention-4 backend for Blackwell
+  #1235" (keys = n_train, here the 30k rows from which the issue reports
+  gains; fp16 as its autocast; the head count is not given: 8).
+* ``vision_d72``: dense non-causal MHA, B=32, S=729, H=16, D=72: the D72 MHA
+  profile of "flashrt/fa4-cute-runtime" (a vision encoder; the page gives no
+  shape: 27x27 patches, 16 heads, a batch of 32 images).
 
 Seeds are 440410 + workload index (the seed style of the pages' benchmark).
 Values are drawn in float32 as N(0, 1) and rounded to the input dtype.
@@ -40,7 +47,7 @@ SEED_BASE = 440410
 
 WORKLOADS = ["dense_257", "varlen_gqa_bias", "video_dit_20480",
              "encoder_d256_seqused", "decode_splitkv", "dense_d64",
-             "local_window_softcap"]
+             "local_window_softcap", "tabpfn_d16", "vision_d72"]
 
 _CHUNK = 1 << 24
 
@@ -238,6 +245,20 @@ def make(name: str, dtype=torch.bfloat16, device="cpu", decode_sk: int = 131072)
         v = _randn((B, S, Hkv, D), g, dtype)
         return Problem(name, "dense", q, k, v, causal=True, softmax_scale=1 / math.sqrt(D),
                        max_seqlen_q=S, max_seqlen_k=S, window=(4095, -1), softcap=50.0)
+    if name == "tabpfn_d16":
+        B, S, H, D = 1, 30000, 8, 16
+        q = _randn((B, S, H, D), g, torch.float16)
+        k = _randn((B, S, H, D), g, torch.float16)
+        v = _randn((B, S, H, D), g, torch.float16)
+        return Problem(name, "dense", q, k, v, softmax_scale=1 / math.sqrt(D),
+                       max_seqlen_q=S, max_seqlen_k=S)
+    if name == "vision_d72":
+        B, S, H, D = 32, 729, 16, 72
+        q = _randn((B, S, H, D), g, dtype)
+        k = _randn((B, S, H, D), g, dtype)
+        v = _randn((B, S, H, D), g, dtype)
+        return Problem(name, "dense", q, k, v, softmax_scale=1 / math.sqrt(D),
+                       max_seqlen_q=S, max_seqlen_k=S)
     raise KeyError(name)
 
 

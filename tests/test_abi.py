@@ -108,6 +108,8 @@ def test_splitkv_host_logic(lib):
     assert 16 <= ns <= 256
     assert ds(8, 1, 2048, 32, 8, 128, 148) <= 2            # short keys
     assert ds(64, 1024, 4096, 32, 32, 128, 148) == 1        # already many units
+    # a short call (8 units of 8 key tiles on 148 SMs): splits of 2 tiles
+    assert ds(1, 128, 1024, 8, 1, 64, 148) == 4
     r = lib.fa_fwd_splitkv(A, A, A, A, A, 1, 1, 16, 4, 2, 128, 0, 0, 0.0, None,
                            None, 0, -1, A, 1 << 20, None)
     assert r == FA_ERR_INVALID

@@ -368,6 +368,10 @@ def test_workload_shapes_match_their_descriptions():
     # 1e4 rounded to bf16
     pad = float(torch.tensor(1e4).to(torch.bfloat16))
     assert float(p.k[0, 968:].float().min()) == pad and float(p.v[1, 968:].float().max()) == pad
+    p = fa_inputs.make("tabpfn_d16")
+    assert tuple(p.q.shape) == (1, 30000, 8, 16) and p.q.dtype == torch.float16
+    p = fa_inputs.make("vision_d72")
+    assert tuple(p.k.shape) == (32, 729, 16, 72) and not p.causal
 
 
 # --------------------------------------------------------------------------

@@ -213,6 +213,19 @@ def test_dense_d64_sampled():
     compare(go, gl, ro, rl, what="dense_d64 sampled")
 
 
+@pytest.mark.parametrize("name,B,H,S", [("tabpfn_d16", 1, 8, 30000), ("vision_d72", 32, 16, 729)])
+def test_narrow_head_dim_workloads_sampled(name, B, H, S):
+    p = fa_inputs.make(name)
+    out, lse = run_dense(p)
+    rows = _sample_rows(np.random.default_rng(4), B, H, [S] * B, 256)
+    ro, rl = oracle.attention_rows(p.q, p.k, p.v, rows, softmax_scale=p.softmax_scale)
+    o = out.float().cpu()
+    l = lse.cpu()
+    go = np.stack([o[b, i, h].numpy() for b, h, i in rows])
+    gl = np.array([float(l[b, h, i]) for b, h, i in rows])
+    compare(go, gl, ro, rl, what=f"{name} sampled")
+
+
 # ---------------------------------------------------------------------------
 # split-KV
 # ---------------------------------------------------------------------------
@@ -434,3 +447,51 @@ def test_watchdog_timeout_is_reported_and_the_device_stays_usable():
     out, lse = run_dense(p)
     ro, rl = ref_dense(p)
     compare(out, lse, ro, rl, what="after the watchdog self-test")
+
+
+# ---------------------------------------------------------------------------
+# CUDA graphs: the library allocates nothing and never synchronises, so a
+# forward captured once replays on new inputs with the same bits as a call
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("D", [16, 64, 128])
+def test_cuda_graph_capture_replays_the_forward(D):
+    p = fa_inputs.random_dense(400 + D, 2, 200, 333, 8, 2, D, causal=True)
+    g = p.to(DEV)
+    q = g.q.clone()
+    out = torch.empty_like(q)
+    lse = torch.empty((2, 8, 200), dtype=torch.float32, device=DEV)
+    fa.fa_fwd(q, g.k, g.v, causal=True, out=out, lse=lse)  # one-time setup outside capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        fa.fa_fwd(q, g.k, g.v, causal=True, out=out, lse=lse)
+    p2 = fa_inputs.random_dense(500 + D, 2, 200, 333, 8, 2, D, causal=True)
+    q.copy_(p2.q.to(DEV))
+    graph.replay()
+    torch.cuda.synchronize()
+    ref_o, ref_l = fa.fa_fwd(q, g.k, g.v, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref_o) and torch.equal(lse, ref_l)
+    ro, rl = oracle.attention(p2.q, p.k, p.v, causal=True, softmax_scale=p.softmax_scale)
+    compare(out, lse, ro, rl, what=f"graph replay D{D}")
+    del graph
+
+
+def test_cuda_graph_capture_of_splitkv_with_a_workspace():
+    p = fa_inputs.random_dense(600, 2, 1, 3000, 8, 2, 128)
+    g = p.to(DEV)
+    ns = 5
+    ws = torch.empty(fa.splitkv_workspace_bytes(2, 1, 8, 128, ns), dtype=torch.uint8, device=DEV)
+    out = torch.empty_like(g.q)
+    lse = torch.empty((2, 8, 1), dtype=torch.float32, device=DEV)
+    fa.fa_fwd_splitkv(g.q, g.k, g.v, num_splits=ns, out=out, lse=lse, workspace=ws)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        fa.fa_fwd_splitkv(g.q, g.k, g.v, num_splits=ns, out=out, lse=lse, workspace=ws)
+    out.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    ro, rl = ref_dense(p)
+    compare(out, lse, ro, rl, what="graph replay split-KV")
+    del graph
