@@ -76,6 +76,8 @@ fa_status encode_map(CUtensorMap *tm, const void *base, int D, int H, long long 
 
 // 3-D map over a [tokens, heads, D] tensor of 16-bit elements with a box of
 // {64 columns, box_h heads, box_t tokens}, 128-byte swizzle, zero fill.
+int kernel_width(int D);
+
 fa_status make_map(CUtensorMap *tm, const void *base, int D, int H, long long tokens, int box_h,
                    int box_t, bool half) {
   const MapKey k{base, tokens, D, H, box_h, box_t, half ? 1 : 0};
@@ -103,7 +105,7 @@ fa_status encode_map(CUtensorMap *tm, const void *base, int D, int H, long long 
   // head dims that are a multiple of 64: 64-column boxes, 128-byte swizzle;
   // narrow ones: 16-column boxes, 32-byte swizzle (the columns past D of the
   // last box read as zero)
-  const bool narrow = D % 64 != 0;
+  const bool narrow = kernel_width(D) % 64 != 0;
   cuuint32_t box[3] = {narrow ? 16u : 64u, (cuuint32_t)box_h, (cuuint32_t)box_t};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = fn(tm, half ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
@@ -135,14 +137,18 @@ int num_sms(int dev) {
 // kernel variants
 // kernel configurations by (16-bit format: bf16 / fp16, modifiers off / on)
 template <bool H, bool M> using Fwd16 = FwdCfg<16, 128, 2, 1, 3, 0, H, false, M>;
+template <bool H, bool M> using Fwd32 = FwdCfg<32, 128, 2, 1, 3, 0, H, false, M>;
 template <bool H, bool M> using Fwd48 = FwdCfg<48, 128, 2, 1, 3, 0, H, false, M>;
 template <bool H, bool M> using Fwd80 = FwdCfg<80, 128, 2, 1, 3, 0, H, false, M>;
+template <bool H, bool M> using Fwd96 = FwdCfg<96, 128, 2, 1, 3, 0, H, false, M>;
 template <bool H, bool M> using Fwd64 = FwdCfg<64, 128, 2, 1, 3, 0, H, false, M>;
 template <bool H, bool M> using Fwd128 = FwdCfg<128, 128, 2, 1, 3, 0, H, false, M>;
 template <bool H, bool M> using Fwd256 = FwdCfg<256, 64, 1, 2, 3, 2, H, false, M>;
 template <bool H, bool M> using Spl16 = FwdCfg<16, 128, 1, 2, 3, 3, H, true, M>;
+template <bool H, bool M> using Spl32 = FwdCfg<32, 128, 1, 2, 3, 3, H, true, M>;
 template <bool H, bool M> using Spl48 = FwdCfg<48, 128, 1, 2, 3, 3, H, true, M>;
 template <bool H, bool M> using Spl80 = FwdCfg<80, 128, 1, 2, 3, 3, H, true, M>;
+template <bool H, bool M> using Spl96 = FwdCfg<96, 128, 1, 2, 3, 3, H, true, M>;
 template <bool H, bool M> using Spl64 = FwdCfg<64, 128, 1, 2, 3, 3, H, true, M>;
 template <bool H, bool M> using Spl128 = FwdCfg<128, 128, 1, 2, 3, 3, H, true, M>;
 template <bool H, bool M> using Spl256 = FwdCfg<256, 64, 1, 2, 2, 2, H, true, M>;
@@ -207,10 +213,20 @@ void apply_mods(Common &c, const fa_mods *m) {
   c.softcap = m->softcap;
 }
 
-// Head dims with a kernel: 64, 128, 256, and the narrow ones served by
-// 16-column-chunk kernels of width 16, 48 or 80 (D = 72 padded to 80).
-bool head_dim_served(int D) {
-  return D == 16 || D == 48 || D == 64 || D == 72 || D == 80 || D == 128 || D == 256;
+// Head dims: every multiple of 8 from 16 to 256.  Each runs in the kernel of
+// the next width up; the tensors keep their own D (row pitch D), the columns
+// past D read as zeros (the loads fill them) and are never stored.  Widths:
+// 64, 128 and 256 with 64-column chunks and a 128-byte swizzle; 16, 32, 48,
+// 80 and 96 with 16-column chunks and a 32-byte swizzle.
+bool head_dim_served(int D) { return D % 8 == 0 && D >= 16 && D <= 256; }
+
+int kernel_width(int D) {
+  if (D == 64 || D == 128 || D == 256) return D;
+  if (D <= 48) return (D + 15) / 16 * 16;  // 16, 32, 48
+  if (D <= 80) return 80;                  // 56, 72, 80
+  if (D <= 96) return 96;                  // 88, 96
+  if (D <= 128) return 128;                // 104 .. 120
+  return 256;                              // 136 .. 248
 }
 
 fa_status validate(const Common &c) {
@@ -219,7 +235,7 @@ fa_status validate(const Common &c) {
     return fail(FA_ERR_INVALID, "B must be >= 0 and Hq, Hkv, D > 0");
   if (c.Hq % c.Hkv != 0) return fail(FA_ERR_INVALID, "Hq (%d) must be a multiple of Hkv (%d)", c.Hq, c.Hkv);
   if (!head_dim_served(c.D))
-    return fail(FA_ERR_UNSUPPORTED, "head_dim %d not served (16, 48, 64, 72, 80, 128 or 256)", c.D);
+    return fail(FA_ERR_UNSUPPORTED, "head_dim %d not served (multiples of 8 from 16 to 256)", c.D);
   if (!c.varlen && (c.Sq < 0 || c.Sk < 0)) return fail(FA_ERR_INVALID, "Sq, Sk must be >= 0");
   if (c.varlen && (c.total_q < 0 || c.total_k < 0 || c.max_q < 0))
     return fail(FA_ERR_INVALID, "total_q, total_k, max_seqlen_q must be >= 0");
@@ -325,18 +341,23 @@ fa_status run_fwd(const Common &c, cudaStream_t st) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return fail(FA_ERR_CUDA, "cudaGetDevice failed");
   FwdParams p;
-  // D <= 128: two Q tiles per CTA, 128-key tiles; D = 256: one Q tile, 64-key tiles
-  const bool wide = c.D == 256;
+  // width <= 128: two Q tiles per CTA, 128-key tiles; 256: one Q tile, 64-key tiles
+  const int w = kernel_width(c.D);
+  const bool wide = w == 256;
   if ((s = fill_params(c, p, wide ? 1 : 2, wide ? 64 : 128, 1, 0x7fffffff)) != FA_OK) return s;
   if (p.num_units == 0) return FA_OK;
   const bool half = c.dt == FA_FP16;
   const bool mods = uses_mods(p);
-  if (c.D == 16) return launch_variant<Fwd16>(p, dev, st, half, mods);
-  if (c.D == 48) return launch_variant<Fwd48>(p, dev, st, half, mods);
-  if (c.D == 72 || c.D == 80) return launch_variant<Fwd80>(p, dev, st, half, mods);
-  if (c.D == 64) return launch_variant<Fwd64>(p, dev, st, half, mods);
-  if (c.D == 128) return launch_variant<Fwd128>(p, dev, st, half, mods);
-  return launch_variant<Fwd256>(p, dev, st, half, mods);
+  switch (w) {
+    case 16: return launch_variant<Fwd16>(p, dev, st, half, mods);
+    case 32: return launch_variant<Fwd32>(p, dev, st, half, mods);
+    case 48: return launch_variant<Fwd48>(p, dev, st, half, mods);
+    case 64: return launch_variant<Fwd64>(p, dev, st, half, mods);
+    case 80: return launch_variant<Fwd80>(p, dev, st, half, mods);
+    case 96: return launch_variant<Fwd96>(p, dev, st, half, mods);
+    case 128: return launch_variant<Fwd128>(p, dev, st, half, mods);
+    default: return launch_variant<Fwd256>(p, dev, st, half, mods);
+  }
 }
 
 template <int D, bool HALF, bool F32OUT>
@@ -391,7 +412,7 @@ fa_status combine(int D, bool half, bool f32out, const float *o_part, const floa
 #undef FA_COMBINE
 }
 
-int splitkv_bn(int D) { return D == 256 ? 64 : 128; }
+int splitkv_bn(int D) { return kernel_width(D) == 256 ? 64 : 128; }
 
 
 // Split-KV forward of a dense problem: the keys are cut into num_splits
@@ -435,18 +456,17 @@ fa_status run_splitkv(const Common &c, int num_splits, void *workspace, size_t w
     p.lse_part = p.o_part + (size_t)ns * rows * D;
   }
   const bool half = c.dt == FA_FP16;
-  if (D == 16)
-    s = launch_variant<Spl16>(p, dev, st, half, uses_mods(p));
-  else if (D == 48)
-    s = launch_variant<Spl48>(p, dev, st, half, uses_mods(p));
-  else if (D == 72 || D == 80)
-    s = launch_variant<Spl80>(p, dev, st, half, uses_mods(p));
-  else if (D == 64)
-    s = launch_variant<Spl64>(p, dev, st, half, uses_mods(p));
-  else if (D == 128)
-    s = launch_variant<Spl128>(p, dev, st, half, uses_mods(p));
-  else
-    s = launch_variant<Spl256>(p, dev, st, half, uses_mods(p));
+  const bool mods = uses_mods(p);
+  switch (kernel_width(D)) {
+    case 16: s = launch_variant<Spl16>(p, dev, st, half, mods); break;
+    case 32: s = launch_variant<Spl32>(p, dev, st, half, mods); break;
+    case 48: s = launch_variant<Spl48>(p, dev, st, half, mods); break;
+    case 64: s = launch_variant<Spl64>(p, dev, st, half, mods); break;
+    case 80: s = launch_variant<Spl80>(p, dev, st, half, mods); break;
+    case 96: s = launch_variant<Spl96>(p, dev, st, half, mods); break;
+    case 128: s = launch_variant<Spl128>(p, dev, st, half, mods); break;
+    default: s = launch_variant<Spl256>(p, dev, st, half, mods); break;
+  }
   if (s != FA_OK || direct) return s;
   return combine(D, half, to_partial, p.o_part, p.lse_part, ns, rows, c.out, c.lse, Hq, Sq, B,
                  st);
@@ -591,7 +611,7 @@ fa_status fa_combine_partials(const float *o_parts, const float *lse_parts, int 
   if (dt != FA_BF16 && dt != FA_FP16) return fail(FA_ERR_INVALID, "dtype must be bf16 or fp16");
   if (B < 0 || Sq < 0 || Hq <= 0) return fail(FA_ERR_INVALID, "B, Sq must be >= 0 and Hq > 0");
   if (!head_dim_served(D))
-    return fail(FA_ERR_UNSUPPORTED, "head_dim %d not served (16, 48, 64, 72, 80, 128 or 256)", D);
+    return fail(FA_ERR_UNSUPPORTED, "head_dim %d not served (multiples of 8 from 16 to 256)", D);
   if (n_parts < 1) return fail(FA_ERR_INVALID, "n_parts must be >= 1");
   const long long rows = (long long)B * Sq * Hq;
   if (rows == 0) return FA_OK;

@@ -374,7 +374,10 @@ struct FwdCfg {
   // or rescales O.  Measured 9-15% slower at D = 16 and 64: the two tiles'
   // softmaxes then run at the same time on the same SMSPs instead of taking
   // turns, and their exponential and FMA work per SMSP does not shrink.
-  static constexpr bool kSepPWanted = false;
+#ifndef FA_SEPARATE_P
+#define FA_SEPARATE_P 0
+#endif
+  static constexpr bool kSepPWanted = FA_SEPARATE_P != 0;
   static constexpr bool kSepP = kSepPWanted && kSplitPV && NQ == 2 && !kSplitS &&
                                 NQ * NS * BN + NQ * ((D + 31) / 32 * 32) + NQ * (BN / 2) <= 512;
   // barrier indices
@@ -895,9 +898,9 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
                                              int t) {
   auto bar = [&](int i) { return sb + C::kBarOff + 8u * i; };
   constexpr int BN = C::BN, D = C::D, NS = C::NS;
-  // row pitch of the output: the tensors' head dim (narrow dims are padded
-  // in the kernel; their padding columns are never stored)
-  const int dO = C::kNarrow ? p.d_out : D;
+  // row pitch of the output: the tensors' head dim (the kernel's D, or less:
+  // the padding columns are never stored)
+  const int dO = p.d_out;
   const int tid = static_cast<int>(threadIdx.x) - 128 * (t + 1);  // tile row == TMEM lane
   const int lane = tid & 31;
   const uint32_t lane_addr = static_cast<uint32_t>(tid & ~31) << 16;
@@ -1219,7 +1222,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
             float *dst = reinterpret_cast<float *>(out_row) + 32 * c;
 #pragma unroll
             for (int e = 0; e < 32; e += 4) {
-              if (C::kNarrow && 32 * c + e >= dO) break;
+              if (32 * c + e >= dO) break;
               float4 w = make_float4(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l,
                                      __uint_as_float(r[e + 2]) * inv_l,
                                      __uint_as_float(r[e + 3]) * inv_l);
@@ -1229,7 +1232,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
             uint16_t *dst = reinterpret_cast<uint16_t *>(out_row) + 32 * c;
 #pragma unroll
             for (int e = 0; e < 32; e += 8) {
-              if (C::kNarrow && 32 * c + e >= dO) break;
+              if (32 * c + e >= dO) break;
               uint4 w;
               w.x = pack2<C::HALF>(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l);
               w.y = pack2<C::HALF>(__uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
@@ -1437,8 +1440,8 @@ __global__ void __launch_bounds__(256) fa_combine_kernel(const float *__restrict
   }
 }
 
-// The same merge for narrow head dims d (a multiple of 8, at most 128): lane
-// l handles the column pairs starting at 2l and 2l + 64.
+// The same merge for head dims d that are not a multiple of 64 (a multiple
+// of 8, at most 256): lane l handles the column pairs starting at 2l + 64k.
 template <bool HALF, bool F32OUT>
 __global__ void __launch_bounds__(256) fa_combine_narrow_kernel(const float *__restrict__ o_part,
                                                                 const float *__restrict__ lse_part,
@@ -1459,35 +1462,41 @@ __global__ void __launch_bounds__(256) fa_combine_narrow_kernel(const float *__r
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
   const float Lse = (m == -INFINITY) ? -INFINITY : m + lg2_approx(z) * 0.69314718055994531f;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  const int c0 = 2 * lane, c1 = 2 * lane + 64;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
   if (m != -INFINITY) {
     for (int s = 0; s < ns; ++s) {
       const float ls = __ldg(lse_part + (long long)s * rows + r);
       if (ls == -INFINITY) continue;
       const float w = ex2_approx((ls - Lse) * L2E);
       const float *src = o_part + ((long long)s * rows + r) * d;
-      if (c0 < d) {
-        const float2 v = __ldg(reinterpret_cast<const float2 *>(src + c0));
-        acc[0] += w * v.x;
-        acc[1] += w * v.y;
-      }
-      if (c1 < d) {
-        const float2 v = __ldg(reinterpret_cast<const float2 *>(src + c1));
-        acc[2] += w * v.x;
-        acc[3] += w * v.y;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int c = 2 * lane + 64 * k;
+        if (c < d) {
+          const float2 v = __ldg(reinterpret_cast<const float2 *>(src + c));
+          acc[2 * k] += w * v.x;
+          acc[2 * k + 1] += w * v.y;
+        }
       }
     }
   }
   if constexpr (F32OUT) {
     float *dst = reinterpret_cast<float *>(out) + r * d;
-    if (c0 < d) *reinterpret_cast<float2 *>(dst + c0) = make_float2(acc[0], acc[1]);
-    if (c1 < d) *reinterpret_cast<float2 *>(dst + c1) = make_float2(acc[2], acc[3]);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int c = 2 * lane + 64 * k;
+      if (c < d) *reinterpret_cast<float2 *>(dst + c) = make_float2(acc[2 * k], acc[2 * k + 1]);
+    }
     if (lane == 0) lse[r] = Lse;
   } else {
     uint16_t *dst = reinterpret_cast<uint16_t *>(out) + r * d;
-    if (c0 < d) *reinterpret_cast<uint32_t *>(dst + c0) = pack2<HALF>(acc[0], acc[1]);
-    if (c1 < d) *reinterpret_cast<uint32_t *>(dst + c1) = pack2<HALF>(acc[2], acc[3]);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int c = 2 * lane + 64 * k;
+      if (c < d) *reinterpret_cast<uint32_t *>(dst + c) = pack2<HALF>(acc[2 * k], acc[2 * k + 1]);
+    }
     if (lane == 0 && lse != nullptr) {
       const long long tok = r / Hq;
       const int h = (int)(r % Hq);

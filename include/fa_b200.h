@@ -33,10 +33,11 @@
  *     synchronises the stream: a call only enqueues work on `stream`
  *     (a cudaStream_t; NULL means the legacy default stream) and returns.
  *   - Element type `dt` applies to q, k, v, out and rel_bias alike.
- *   - head_dim D must be 16, 48, 64, 72, 80, 128 or 256 ("FlashAttention-4
- *     backend for Blackwell #1235" uses head dims 16 and 64,
- *     "flashrt/fa4-cute-runtime" the D48/D72/D128 family and D256); Hq must
- *     be a multiple of Hkv; query head h reads K/V head h / (Hq / Hkv).
+ *   - head_dim D must be a multiple of 8 from 16 to 256 ("FlashAttention-4
+ *     backend for Blackwell #1235" uses head dims 16 and 64 and gives FA4's
+ *     range on SM100 in steps of 8; "flashrt/fa4-cute-runtime" the
+ *     D48/D72/D128 family and D256); Hq must be a multiple of Hkv; query
+ *     head h reads K/V head h / (Hq / Hkv).
  *   - q, k, v, out and rel_bias must be 16-byte aligned and contiguous in the
  *     documented layout.  cu_seqlens and seqused_k are device int32 arrays.
  *   - softmax_scale <= 0 selects 1 / sqrt(D).
@@ -62,7 +63,7 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID = 1,        /* malformed arguments (null, shape, alignment) */
-  FA_ERR_UNSUPPORTED = 2,    /* well-formed but not served (e.g. D = 96)    */
+  FA_ERR_UNSUPPORTED = 2,    /* well-formed but not served (e.g. D = 100)   */
   FA_ERR_CUDA = 3,           /* a CUDA runtime call or launch failed         */
   FA_ERR_WORKSPACE = 4,      /* split-KV workspace missing or too small      */
   FA_ERR_DEVICE_TIMEOUT = 5  /* a kernel gave up waiting (see below)         */

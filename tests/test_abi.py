@@ -55,9 +55,11 @@ def _fwd(lib, q=A, k=A, v=A, out=A, lse=A, B=1, Sq=16, Sk=16, Hq=4, Hkv=2, D=128
 
 
 def test_validation_statuses(lib):
-    assert _fwd(lib, D=96) == FA_ERR_UNSUPPORTED
-    assert _fwd(lib, D=32) == FA_ERR_UNSUPPORTED
-    assert _fwd(lib, D=192) == FA_ERR_UNSUPPORTED
+    # head dims: multiples of 8 from 16 to 256
+    assert _fwd(lib, D=8) == FA_ERR_UNSUPPORTED
+    assert _fwd(lib, D=100) == FA_ERR_UNSUPPORTED
+    assert _fwd(lib, D=264) == FA_ERR_UNSUPPORTED
+    assert _fwd(lib, D=12) == FA_ERR_UNSUPPORTED
     assert _fwd(lib, Hq=6, Hkv=4) == FA_ERR_INVALID
     assert _fwd(lib, dt=7) == FA_ERR_INVALID
     assert _fwd(lib, q=None) == FA_ERR_INVALID
@@ -91,7 +93,7 @@ def test_varlen_validation(lib):
     r = lib.fa_fwd_varlen(A, A, A, A, A, None, None, None, 2, 8, 8, 16, 16, 4, 2,
                           128, 0, 0, 0.0, None, 0, None)
     assert r == FA_ERR_INVALID  # cu_seqlens missing
-    r = lib.fa_fwd_varlen(A, A, A, A, A, A, A, P, 2, 8, 8, 16, 16, 4, 2, 96, 0, 0,
+    r = lib.fa_fwd_varlen(A, A, A, A, A, A, A, P, 2, 8, 8, 16, 16, 4, 2, 100, 0, 0,
                           0.0, None, 0, None)
     assert r == FA_ERR_UNSUPPORTED
 
@@ -132,13 +134,13 @@ def test_shard_partial_and_combine_validation(lib):
     sp = lib.fa_fwd_shard_partial
     args = lambda D=128, lse=A, ns=1: (A, A, A, A, lse, 1, 1, 16, 4, 2, D, 0, 0, 0.0,  # noqa: E731
                                        None, None, None, 0, None, ns, None, 0, None)
-    assert sp(*args(D=96)) == FA_ERR_UNSUPPORTED
+    assert sp(*args(D=100)) == FA_ERR_UNSUPPORTED
     assert sp(*args(lse=None)) == FA_ERR_INVALID
     assert sp(*args(ns=-1)) == FA_ERR_INVALID
     # combine: part count, head dim, dtype and alignment are checked first
     cp = lib.fa_combine_partials
     assert cp(A, A, 0, 1, 1, 4, 128, 0, A, A, None) == FA_ERR_INVALID
-    assert cp(A, A, 2, 1, 1, 4, 96, 0, A, A, None) == FA_ERR_UNSUPPORTED
+    assert cp(A, A, 2, 1, 1, 4, 100, 0, A, A, None) == FA_ERR_UNSUPPORTED
     assert cp(A, A, 2, 1, 1, 4, 128, 7, A, A, None) == FA_ERR_INVALID
     assert cp(MIS, A, 2, 1, 1, 4, 128, 0, A, A, None) == FA_ERR_INVALID
     assert cp(A, A, 2, 1, 1, 4, 128, 0, None, A, None) == FA_ERR_INVALID

@@ -346,7 +346,7 @@ def test_many_batches_beyond_grid_y_limit():
 
 
 def test_invalid_arguments_raise_and_write_nothing():
-    q = torch.randn(1, 16, 4, 96, device=DEV, dtype=torch.bfloat16)
+    q = torch.randn(1, 16, 4, 100, device=DEV, dtype=torch.bfloat16)  # not a multiple of 8
     with pytest.raises(fa.FAError) as e:
         fa.fa_fwd(q, q, q)
     assert e.value.name == "FA_ERR_UNSUPPORTED"
@@ -495,3 +495,33 @@ def test_cuda_graph_capture_of_splitkv_with_a_workspace():
     ro, rl = ref_dense(p)
     compare(out, lse, ro, rl, what="graph replay split-KV")
     del graph
+
+
+# ---------------------------------------------------------------------------
+# every head dim the library serves: multiples of 8 from 16 to 256, each in
+# the kernel of the next width up (padding columns read as zeros, never stored)
+# ---------------------------------------------------------------------------
+SWEEP_D = [16, 24, 32, 40, 48, 56, 64, 72, 88, 96, 104, 120, 128, 136, 192, 248, 256]
+
+
+@pytest.mark.parametrize("D", SWEEP_D)
+def test_head_dim_sweep_dense_causal_gqa(D):
+    p = fa_inputs.random_dense(700 + D, 1, 200, 333, 8, 2, D, causal=True)
+    out, lse = run_dense(p)
+    ro, rl = ref_dense(p)
+    compare(out, lse, ro, rl, what=f"sweep dense D{D}")
+
+
+@pytest.mark.parametrize("D", [24, 40, 56, 88, 120, 136])
+def test_head_dim_sweep_varlen_bias_and_splitkv(D):
+    p = fa_inputs.random_varlen(800 + D, [0, 130, 257, 1], [5, 300, 257, 1], Hq=8, Hkv=2, D=D,
+                                causal=True, bias_extent=128)
+    out, lse = run_varlen(p)
+    ro, rl = ref_varlen(p)
+    compare(out, lse, ro, rl, what=f"sweep varlen bias D{D}")
+    q = fa_inputs.random_dense(900 + D, 2, 1, 1500, 8, 2, D)
+    g = q.to(DEV)
+    out, lse = fa.fa_fwd_splitkv(g.q, g.k, g.v, num_splits=3)
+    torch.cuda.synchronize()
+    ro, rl = ref_dense(q)
+    compare(out, lse, ro, rl, what=f"sweep split-KV D{D}")
