@@ -897,7 +897,7 @@ template <class C>
 __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, uint32_t tmem,
                                              int t) {
   auto bar = [&](int i) { return sb + C::kBarOff + 8u * i; };
-  constexpr int BN = C::BN, D = C::D, NS = C::NS;
+  constexpr int BN = C::BN, NS = C::NS;
   // row pitch of the output: the tensors' head dim (the kernel's D, or less:
   // the padding columns are never stored)
   const int dO = p.d_out;
