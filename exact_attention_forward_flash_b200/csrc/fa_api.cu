@@ -297,6 +297,9 @@ fa_status fill_params(const Common &c, FwdParams &p, int nq, int bn, int num_spl
   p.rel_bias = static_cast<const uint16_t *>(c.rel_bias);
   p.R = c.rel_bias ? c.R : 0;
   p.d_out = c.D;
+  // 32-byte epilogue stores: the output base and every row 32-byte aligned
+  // (rows of 16-bit outputs hold D * 2 bytes, fp32 partials D * 4)
+  p.st32 = ((reinterpret_cast<uintptr_t>(c.out) & 31) == 0 && c.D % 16 == 0) ? 1 : 0;
   p.B = c.B;
   p.Sq = c.Sq;
   p.Sk = c.Sk;
@@ -455,6 +458,8 @@ fa_status run_splitkv(const Common &c, int num_splits, void *workspace, size_t w
     p.o_part = static_cast<float *>(workspace);
     p.lse_part = p.o_part + (size_t)ns * rows * D;
   }
+  // fp32 partial rows hold D * 4 bytes (a multiple of 32): only the base counts
+  p.st32 = (reinterpret_cast<uintptr_t>(p.o_part) & 31) == 0 ? 1 : 0;
   const bool half = c.dt == FA_FP16;
   const bool mods = uses_mods(p);
   switch (kernel_width(D)) {

@@ -133,6 +133,7 @@ struct FwdParams {
   const uint16_t *rel_bias;      // nullptr or [tok, Hq, R]
   int R;
   int d_out;         // head dim of the tensors (the kernel's D, or less with zero padding)
+  int st32;          // 1: output rows are 32-byte aligned (32-byte stores in the epilogue)
   int B, Sq, Sk, Hq, Hkv, G, P, lgP, n_groups;
   int total_q;
   int n_mblk;        // CTA tiles per (batch, head group, split)
@@ -1220,6 +1221,23 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
         if (valid) {
           if constexpr (C::PARTIAL) {
             float *dst = reinterpret_cast<float *>(out_row) + 32 * c;
+            if (p.st32) {  // 8 columns per 32-byte store
+#pragma unroll
+              for (int e = 0; e < 32; e += 8) {
+                if (32 * c + e >= dO) break;
+                uint4 a, b;
+                a.x = __float_as_uint(__uint_as_float(r[e]) * inv_l);
+                a.y = __float_as_uint(__uint_as_float(r[e + 1]) * inv_l);
+                a.z = __float_as_uint(__uint_as_float(r[e + 2]) * inv_l);
+                a.w = __float_as_uint(__uint_as_float(r[e + 3]) * inv_l);
+                b.x = __float_as_uint(__uint_as_float(r[e + 4]) * inv_l);
+                b.y = __float_as_uint(__uint_as_float(r[e + 5]) * inv_l);
+                b.z = __float_as_uint(__uint_as_float(r[e + 6]) * inv_l);
+                b.w = __float_as_uint(__uint_as_float(r[e + 7]) * inv_l);
+                stg_v8(dst + e, a, b);
+              }
+              continue;
+            }
 #pragma unroll
             for (int e = 0; e < 32; e += 4) {
               if (32 * c + e >= dO) break;
@@ -1230,6 +1248,23 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
             }
           } else {
             uint16_t *dst = reinterpret_cast<uint16_t *>(out_row) + 32 * c;
+            if (p.st32) {  // 16 columns per 32-byte store
+#pragma unroll
+              for (int e = 0; e < 32; e += 16) {
+                if (32 * c + e >= dO) break;
+                uint4 a, b;
+                a.x = pack2<C::HALF>(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l);
+                a.y = pack2<C::HALF>(__uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
+                a.z = pack2<C::HALF>(__uint_as_float(r[e + 4]) * inv_l, __uint_as_float(r[e + 5]) * inv_l);
+                a.w = pack2<C::HALF>(__uint_as_float(r[e + 6]) * inv_l, __uint_as_float(r[e + 7]) * inv_l);
+                b.x = pack2<C::HALF>(__uint_as_float(r[e + 8]) * inv_l, __uint_as_float(r[e + 9]) * inv_l);
+                b.y = pack2<C::HALF>(__uint_as_float(r[e + 10]) * inv_l, __uint_as_float(r[e + 11]) * inv_l);
+                b.z = pack2<C::HALF>(__uint_as_float(r[e + 12]) * inv_l, __uint_as_float(r[e + 13]) * inv_l);
+                b.w = pack2<C::HALF>(__uint_as_float(r[e + 14]) * inv_l, __uint_as_float(r[e + 15]) * inv_l);
+                stg_v8(dst + e, a, b);
+              }
+              continue;
+            }
 #pragma unroll
             for (int e = 0; e < 32; e += 8) {
               if (32 * c + e >= dO) break;
