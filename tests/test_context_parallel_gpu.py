@@ -88,6 +88,15 @@ def test_causal_bias_seqused_shards(D):
     compare(out, lse, ro, rl, what=f"cp causal bias seqused D={D}")
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_fp16_gqa_shards_with_local_splits(D):
+    p = fa_inputs.random_dense(95 + D, 2, 17, 2500, 16, 2, D, dtype=torch.float16, causal=True,
+                               bias_extent=256)
+    out, lse = sharded(p, 3, num_splits=4)
+    ro, rl = ref(p)
+    compare(out, lse, ro, rl, what=f"cp fp16 D={D}")
+
+
 def test_window_softcap_shards():
     p = fa_inputs.random_dense(90, 2, 64, 2000, 8, 2, 128, causal=True, q_std=3.0)
     out, lse = sharded(p, 4, num_splits=2, window=(500, 0), softcap=8.0)

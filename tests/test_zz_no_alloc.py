@@ -35,7 +35,7 @@ def _static_call(lib, q, k, v, out, lse, num_splits, causal=False, seqused=None)
         num_splits, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
-@pytest.mark.parametrize("D,ns", [(128, 0), (128, 9), (256, 5)])
+@pytest.mark.parametrize("D,ns", [(128, 0), (128, 9), (256, 5), (72, 4), (40, 0)])
 def test_static_matches_workspace_entry_twice(D, ns):
     lib = fa.load_library()
     probs = [fa_inputs.random_dense(500 + D + s, 4, 2, 3000, 16, 4, D, causal=True)
