@@ -5,6 +5,13 @@ for bf16 and fp16 outputs; on the LSE, |dLSE| <= 1e-3 * max(1, |LSE|).  The
 relative RMS error of O (<= 1e-2) is also checked, because with N(0,1) inputs
 and long key ranges |O| is so small that the absolute gates say little.
 Rows with no admissible key must give O == 0 exactly and LSE == -inf.
+
+The max-abs bound is taken on top of the output type's own rounding: an
+element may differ from the fp64 reference by 1e-2 plus half a unit in the
+last place of the reference in that type.  Where |O| >= 4 a bf16 half-ulp is
+already 0.0156, so the exactly rounded result itself would exceed a bare
+1e-2 (rows that see a handful of keys under a causal mask reach such |O|);
+for |O| well below 1 the added term is negligible.
 """
 import math
 
@@ -23,17 +30,28 @@ def to_np(t):
     return np.asarray(t, dtype=np.float64)
 
 
+def half_ulp(ref, mantissa_bits):
+    """Half a unit in the last place of |ref| in a float type with the given
+    explicit mantissa bits (7 for bf16, 10 for fp16); 0 where ref is 0."""
+    a = np.abs(ref)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, 2.0 ** (e - mantissa_bits - 1), 0.0)
+
+
 def compare(out, lse, ref_o, ref_l, *, max_abs=MAX_ABS, mean_abs=MEAN_ABS,
             lse_rel=LSE_REL, rel_rms=REL_RMS, what=""):
     stats = {}
     if out is not None:
+        bits = 10 if isinstance(out, torch.Tensor) and out.dtype == torch.float16 else 7
         o = to_np(out).reshape(ref_o.shape)
         ref_o = np.asarray(ref_o, dtype=np.float64)
         err = np.abs(o - ref_o)
         stats["max_abs"] = float(err.max()) if err.size else 0.0
         stats["mean_abs"] = float(err.mean()) if err.size else 0.0
         assert np.isfinite(o).all(), f"{what}: non-finite output"
-        assert stats["max_abs"] <= max_abs, f"{what}: {stats}"
+        over = err - (max_abs + half_ulp(ref_o, bits))
+        stats["max_over_bound"] = float(over.max()) if err.size else 0.0
+        assert stats["max_over_bound"] <= 0.0, f"{what}: {stats}"
         assert stats["mean_abs"] <= mean_abs, f"{what}: {stats}"
         nrm = float(np.sqrt((ref_o ** 2).sum()))
         if nrm > 0:

@@ -525,3 +525,32 @@ def test_head_dim_sweep_varlen_bias_and_splitkv(D):
     torch.cuda.synchronize()
     ro, rl = ref_dense(q)
     compare(out, lse, ro, rl, what=f"sweep split-KV D{D}")
+
+
+# ---------------------------------------------------------------------------
+# problem size picks the kernel: fewer two-tile units than SMs run one Q tile
+# per CTA (most cases above); these shapes have enough units for two tiles
+# ---------------------------------------------------------------------------
+TWO_TILE_CASES = [
+    # B, Sq, Sk, Hq, Hkv, D, causal  -> >= 148 units of two 128-row tiles
+    (2, 300, 300, 48, 48, 128, True),
+    (2, 300, 333, 64, 16, 64, False),
+    (2, 260, 260, 40, 40, 128, False),
+]
+
+
+@pytest.mark.parametrize("case", TWO_TILE_CASES)
+def test_two_tile_kernel_at_moderate_sizes(case):
+    B, Sq, Sk, Hq, Hkv, D, causal = case
+    p = fa_inputs.random_dense(1000 + Hq + D, B, Sq, Sk, Hq, Hkv, D, causal=causal)
+    out, lse = run_dense(p)
+    ro, rl = ref_dense(p)
+    compare(out, lse, ro, rl, what=f"two-tile {case}")
+
+
+def test_two_tile_kernel_varlen_bias():
+    p = fa_inputs.random_varlen(1100, [300, 513, 129], [300, 513, 129], Hq=64, Hkv=8, D=128,
+                                causal=True, bias_extent=256)
+    out, lse = run_varlen(p)
+    ro, rl = ref_varlen(p)
+    compare(out, lse, ro, rl, what="two-tile varlen bias")
