@@ -147,7 +147,12 @@ template <bool H, bool M> using Fwd256 = FwdCfg<256, 64, 1, 2, 3, 2, H, false, M
 // one Q tile per CTA with a double-buffered S: each unit runs at the
 // softmax's own rate instead of sharing its SMSPs with a second tile; for
 // problems with fewer two-tile units than SMs (latency-bound calls)
+template <bool H, bool M> using Lat16 = FwdCfg<16, 128, 1, 2, 3, 3, H, false, M>;
+template <bool H, bool M> using Lat32 = FwdCfg<32, 128, 1, 2, 3, 3, H, false, M>;
+template <bool H, bool M> using Lat48 = FwdCfg<48, 128, 1, 2, 3, 3, H, false, M>;
 template <bool H, bool M> using Lat64 = FwdCfg<64, 128, 1, 2, 3, 3, H, false, M>;
+template <bool H, bool M> using Lat80 = FwdCfg<80, 128, 1, 2, 3, 3, H, false, M>;
+template <bool H, bool M> using Lat96 = FwdCfg<96, 128, 1, 2, 3, 3, H, false, M>;
 template <bool H, bool M> using Lat128 = FwdCfg<128, 128, 1, 2, 3, 3, H, false, M>;
 template <bool H, bool M> using Spl16 = FwdCfg<16, 128, 1, 2, 3, 3, H, true, M>;
 template <bool H, bool M> using Spl32 = FwdCfg<32, 128, 1, 2, 3, 3, H, true, M>;
@@ -356,11 +361,18 @@ fa_status run_fwd(const Common &c, cudaStream_t st) {
   if (p.num_units == 0) return FA_OK;
   const bool half = c.dt == FA_FP16;
   const bool mods = uses_mods(p);
-  if ((w == 64 || w == 128) && p.num_units < num_sms(dev)) {
+  if (w <= 128 && p.num_units < num_sms(dev)) {
     // fewer two-tile units than SMs: one tile per CTA, twice the units
     if ((s = fill_params(c, p, 1, 128, 1, 0x7fffffff)) != FA_OK) return s;
-    return w == 64 ? launch_variant<Lat64>(p, dev, st, half, mods)
-                   : launch_variant<Lat128>(p, dev, st, half, mods);
+    switch (w) {
+      case 16: return launch_variant<Lat16>(p, dev, st, half, mods);
+      case 32: return launch_variant<Lat32>(p, dev, st, half, mods);
+      case 48: return launch_variant<Lat48>(p, dev, st, half, mods);
+      case 64: return launch_variant<Lat64>(p, dev, st, half, mods);
+      case 80: return launch_variant<Lat80>(p, dev, st, half, mods);
+      case 96: return launch_variant<Lat96>(p, dev, st, half, mods);
+      default: return launch_variant<Lat128>(p, dev, st, half, mods);
+    }
   }
   switch (w) {
     case 16: return launch_variant<Fwd16>(p, dev, st, half, mods);

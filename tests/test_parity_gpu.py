@@ -536,6 +536,9 @@ TWO_TILE_CASES = [
     (2, 300, 300, 48, 48, 128, True),
     (2, 300, 333, 64, 16, 64, False),
     (2, 260, 260, 40, 40, 128, False),
+    (2, 300, 300, 48, 48, 16, True),
+    (2, 300, 333, 64, 16, 72, False),
+    (2, 260, 260, 40, 40, 48, True),
 ]
 
 
