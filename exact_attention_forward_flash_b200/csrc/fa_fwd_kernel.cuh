@@ -20,7 +20,7 @@
 //               BN keys through shared-memory rings (separate K and V rings,
 //               or one ring that K and V tiles take in turn).
 //   warp 1      MMA issuer (the warp's elected lane): S = Q K^T (SS form, both operands
-//               K-major in 128B-swizzled shared memory) into tensor memory,
+//               K-major in swizzled shared memory) into tensor memory,
 //               and O += P V (TS form: P read from tensor memory where it
 //               overwrites S, V MN-major in shared memory).  Also owns the
 //               tensor-memory allocation.
@@ -35,7 +35,17 @@
 //
 // A Q tile holds 128 packed rows: P consecutive query heads that share one
 // K/V head (P = Hq/Hkv when that divides 128, else 1) at 128/P consecutive
-// positions, loaded with one 3-D TMA box {64, P, 128/P} per 64 columns.
+// positions, loaded with one 3-D TMA box {64, P, 128/P} per 64 columns
+// (128-byte swizzle) or, for head dims that are not a multiple of 64, one
+// {16, P, 128/P} box per 16 columns (32-byte swizzle).  The kernel width D
+// may exceed the tensors' head dim: the loads fill the extra columns with
+// zeros and the epilogue stores only the tensors' columns.
+//
+// Configurations (FwdCfg<D, BN, NQ, NS, KST, VST, HALF, PARTIAL, MODS>): two
+// Q tiles per CTA with one S buffer each (throughput), one Q tile with a
+// double-buffered S (latency-bound calls, D = 256, and the split-KV partial
+// kernels, which write normalised fp32 partials for the merge kernel), and,
+// for each, a MODS kernel that adds the left window bound and the soft-cap.
 //
 // Every wait is bounded (see mbar_wait); a role that gives up records the
 // timeout in g_fa_error, drains what it has in flight, and leaves its loops.
