@@ -14,8 +14,9 @@ def pytest_configure(config):
 
 
 def pytest_collection_modifyitems(config, items):
-    """GPU tests fail loudly on a GPU machine without the library; on a CPU-only
-    box they are skipped (only when ``-m gpu`` was not explicitly asked for)."""
+    """GPU tests fail loudly on a machine with a GPU but without the library;
+    on a CPU-only machine they are skipped (only when ``-m gpu`` was not
+    explicitly asked for)."""
     try:
         import torch
         has_gpu = torch.cuda.is_available()
