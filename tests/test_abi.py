@@ -145,3 +145,18 @@ def test_shard_partial_and_combine_validation(lib):
     assert cp(MIS, A, 2, 1, 1, 4, 128, 0, A, A, None) == FA_ERR_INVALID
     assert cp(A, A, 2, 1, 1, 4, 128, 0, None, A, None) == FA_ERR_INVALID
     assert cp(A, A, 2, 0, 1, 4, 128, 0, A, A, None) == FA_OK  # no rows: nothing to do
+
+
+def test_default_splits_properties(lib):
+    ds = lib.fa_splitkv_default_splits
+    rng = __import__("random").Random(5)
+    for _ in range(500):
+        B, Sq = rng.randint(1, 64), rng.choice([1, 1, 4, 37, 128, 1024])
+        Hkv = rng.choice([1, 2, 4, 8, 32])
+        Hq = Hkv * rng.choice([1, 2, 4, 8])
+        D = rng.choice([16, 64, 72, 128, 256])
+        Sk = rng.randint(1, 300000)
+        ns = ds(B, Sq, Sk, Hq, Hkv, D, 148)
+        bn = 64 if D > 128 else 128
+        assert 1 <= ns <= 256
+        assert ns <= max(1, -(-Sk // (2 * bn)))  # every split holds at least two key tiles

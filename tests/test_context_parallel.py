@@ -133,3 +133,45 @@ def test_two_gloo_ranks_exchange_partials_that_merge_to_the_full_result():
         np.testing.assert_allclose(lse, ref_l.numpy(), rtol=0, atol=1e-12)
         np.testing.assert_allclose(o, ref_o.numpy(), rtol=0, atol=1e-12)
     np.testing.assert_array_equal(res[0][1], res[1][1])
+
+
+# ---------------------------------------------------------------------------
+# property checks of the planner over random sizes
+# ---------------------------------------------------------------------------
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=300, deadline=None)
+@given(k_len=st.integers(0, 1 << 20), world=st.integers(1, 64),
+       align=st.sampled_from([1, 8, 64, 128, 256]))
+def test_shard_bounds_properties(k_len, world, align):
+    shards = [shard_bounds(k_len, world, r, align=align) for r in range(world)]
+    pos = 0
+    for start, length, after in shards:
+        assert start == pos and length >= 0 and after == k_len - start - length
+        pos += length
+    assert pos == k_len
+    blocks = [-(-n // align) for _, n, _ in shards]
+    assert max(blocks) - min(blocks) <= 1
+    # only the last non-empty shard may hold a partial block
+    nonempty = [n for _, n, _ in shards if n]
+    assert all(n % align == 0 for n in nonempty[:-1])
+
+
+@settings(max_examples=300, deadline=None)
+@given(data=st.data())
+def test_shard_seqused_properties(data):
+    world = data.draw(st.integers(1, 9))
+    padded = data.draw(st.integers(0, 5000))
+    used = data.draw(st.lists(st.integers(0, padded), min_size=1, max_size=6))
+    total_used = [0] * len(used)
+    for r in range(world):
+        start, length, _ = shard_bounds(padded, world, r)
+        loc, after = shard_seqused(used, start, length)
+        for b, n in enumerate(used):
+            assert 0 <= loc[b] <= length and after[b] >= 0
+            # valid keys before, in and after the shard add up to all of them
+            before = min(max(n, 0), start)
+            assert before + loc[b] + after[b] == n
+            total_used[b] += loc[b]
+    assert total_used == used
