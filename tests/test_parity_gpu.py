@@ -557,3 +557,29 @@ def test_two_tile_kernel_varlen_bias():
     out, lse = run_varlen(p)
     ro, rl = ref_varlen(p)
     compare(out, lse, ro, rl, what="two-tile varlen bias")
+
+
+def test_two_tile_kernel_fp16_varlen_bias():
+    p = fa_inputs.random_varlen(1200, [300, 513, 129], [300, 513, 129], Hq=64, Hkv=8, D=128,
+                                dtype=torch.float16, causal=True, bias_extent=256)
+    out, lse = run_varlen(p)
+    ro, rl = ref_varlen(p)
+    compare(out, lse, ro, rl, what="two-tile fp16 varlen bias")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_one_tile_kernel_fp16_varlen_bias(D):
+    p = fa_inputs.random_varlen(1300 + D, [0, 77, 300], [5, 200, 300], Hq=8, Hkv=2, D=D,
+                                dtype=torch.float16, causal=True, bias_extent=128)
+    out, lse = run_varlen(p)
+    ro, rl = ref_varlen(p)
+    compare(out, lse, ro, rl, what=f"one-tile fp16 varlen bias D{D}")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_two_tile_modifier_kernel(D):
+    # >= 148 two-tile units, left window + soft-cap: the two-tile MODS kernel
+    p = fa_inputs.random_dense(1400 + D, 2, 300, 300, 48, 48, D, causal=True, q_std=3.0)
+    out, lse = run_dense(p, window=(90, -1), softcap=6.0)
+    ro, rl = ref_dense(p, window=(90, -1), softcap=6.0)
+    compare(out, lse, ro, rl, what=f"two-tile window+softcap D{D}")
