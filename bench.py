@@ -229,8 +229,30 @@ class Runner:
                              lse=self.lse, window=p.window, softcap=p.softcap)
 
 
+class nvtx_range:
+    """A named NVTX range around a timed region, so that a profiler run can
+    select it (ncu --nvtx); nothing when NVTX is unavailable."""
+
+    def __init__(self, name: str):
+        self.name, self.on = name, False
+
+    def __enter__(self):
+        try:
+            import torch
+            torch.cuda.nvtx.range_push(self.name)
+            self.on = True
+        except Exception:
+            self.on = False
+        return self
+
+    def __exit__(self, *exc):
+        if self.on:
+            import torch
+            torch.cuda.nvtx.range_pop()
+
+
 def time_steps(step, steps: int, warmup: int, dist_on: bool, device_index: int,
-               flush=None):
+               flush=None, label: str = "timed steps"):
     """W untimed steps, then K steps between barrier + synchronize; returns
     (total ms over K, mean per-step ms from per-step events, clocks).
 
@@ -248,7 +270,7 @@ def time_steps(step, steps: int, warmup: int, dist_on: bool, device_index: int,
     if dist_on:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(device_index) as clk:
+    with ClockSampler(device_index) as clk, nvtx_range(label):
         t0.record()
         for a, b in evs:
             if flush is not None:
@@ -324,12 +346,13 @@ def time_e2e(p, p_cpu, splits: int, steps: int, dist_on: bool, world: int, unit:
     if dist_on:
         dist.barrier()
     torch.cuda.synchronize()
-    t0.record(s_in)
-    for k in range(steps):
-        step(k)
-    s_in.wait_stream(s_out)
-    t1.record(s_in)
-    torch.cuda.synchronize()
+    with nvtx_range("end to end"):
+        t0.record(s_in)
+        for k in range(steps):
+            step(k)
+        s_in.wait_stream(s_out)
+        t1.record(s_in)
+        torch.cuda.synchronize()
     if dist_on:
         dist.barrier()
     total = max_over_ranks(t0.elapsed_time(t1), dist_on)
@@ -392,8 +415,12 @@ def time_short_calls(dev, n_calls: int = 2000, per_graph: int = 100, replays: in
         return {"eager_us_per_call": round(eager_us, 2), "graph_us_per_call": round(graph_us, 2),
                 "graph_tflops": round(p.flops() / (graph_us * 1e-6) / 1e12, 2)}
 
+    with nvtx_range("short calls: fa_fwd"):
+        plain_res = measure(plain)
+    with nvtx_range("short calls: fa_fwd_splitkv"):
+        split_res = measure(split)
     return {"shape": "dense B=1 Sq=128 Sk=1024 Hq=8 Hkv=1 D=64 fp16",
-            "fa_fwd": measure(plain), "fa_fwd_splitkv": dict(measure(split), num_splits=ns)}
+            "fa_fwd": plain_res, "fa_fwd_splitkv": dict(split_res, num_splits=ns)}
 
 
 def max_over_ranks(x: float, dist_on: bool) -> float:
@@ -514,7 +541,7 @@ def main():
     if main_small:
         flush_buf = torch.empty(4 * l2_bytes, dtype=torch.uint8, device=dev)
     total_ms, per_ms, clocks = time_steps(run, a.steps, a.warmup, dist_on, local,
-                                          flush=flush_buf)
+                                          flush=flush_buf, label=f"timed steps: {a.workload}")
     if main_small:
         total_ms = per_ms * a.steps  # the flush between steps is not the workload's time
     total_ms = max_over_ranks(total_ms, dist_on)
@@ -543,7 +570,8 @@ def main():
             if small and flush_buf is None:
                 flush_buf = torch.empty(4 * l2_bytes, dtype=torch.uint8, device=dev)
             tt, pm, ck = time_steps(r, k_steps, max(3, a.warmup), dist_on, local,
-                                    flush=flush_buf if small else None)
+                                    flush=flush_buf if small else None,
+                                    label=f"timed steps: {name}")
             if small:
                 tt = pm * k_steps  # the flush between steps is not the workload's time
             tt = max_over_ranks(tt, dist_on)
