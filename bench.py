@@ -261,6 +261,10 @@ def time_steps(step, steps: int, warmup: int, dist_on: bool, device_index: int,
     (their time is then the per-step event mean, cold L2)."""
     import torch
     import torch.distributed as dist
+    # NVML is initialised before the warm-up, so that its first
+    # initialisation (a host stall with the device idle) never sits between
+    # the warm-up and the timed region.
+    sampler = ClockSampler(device_index)
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
@@ -270,7 +274,7 @@ def time_steps(step, steps: int, warmup: int, dist_on: bool, device_index: int,
     if dist_on:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(device_index) as clk, nvtx_range(label):
+    with sampler as clk, nvtx_range(label):
         t0.record()
         for a, b in evs:
             if flush is not None:
