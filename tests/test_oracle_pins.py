@@ -457,3 +457,66 @@ def test_softcap_saturates_and_vanishes_in_the_limit():
     z = math.exp(0.5) + math.exp(-0.25)
     np.testing.assert_allclose(out[0, 0], [math.exp(0.5) / z, math.exp(-0.25) / z], atol=1e-12)
     assert lse[0, 0] == pytest.approx(math.log(z), abs=1e-12)
+
+
+def _dtanh(x):
+    """tanh in decimal arithmetic from its exponential definition."""
+    e = (2 * x).exp()
+    return (e - 1) / (e + 1)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("window", [(-1, -1), (1, -1), (2, 0), (-1, 1), (0, 0)])
+@pytest.mark.parametrize("softcap", [0.0, 1.5])
+def test_dense_modifiers_seqused_and_ranges_high_precision(causal, window, softcap):
+    """Brute force in 50-digit decimals on the dense entry: seqused_k sets each
+    sequence's k_len (and so the diagonal), keys are dropped by the causal,
+    left and right distance bounds, the cap maps s to c*tanh(s/c) before the
+    bias is added, and a key range returns the softmax over its keys only.
+    Shapes have Sq != Sk, GQA, and rows that every key misses."""
+    getcontext().prec = 50
+    rng = np.random.default_rng(100 + 10 * causal + 3 * window[0] + window[1] + int(softcap))
+    B, Sq, Sk, Hq, Hkv, D, R = 2, 3, 6, 4, 2, 4, 4
+    seqused = [4, 6]
+    scale = 0.9
+    q = (rng.standard_normal((B, Sq, Hq, D)) * 0.8).astype(np.float32)
+    k = (rng.standard_normal((B, Sk, Hkv, D)) * 0.8).astype(np.float32)
+    v = rng.standard_normal((B, Sk, Hkv, D)).astype(np.float32)
+    k[0, 4:] = 1e4  # padding past seqused_k must never be read
+    v[0, 4:] = 1e4
+    rb = rng.standard_normal((B * Sq, Hq, R)).astype(np.float32)
+    cap = Decimal(softcap)
+    left, right = window
+    for kv_range in (None, (1, 4)):
+        kw = dict(seqused_k=np.array(seqused, np.int32), causal=causal, softmax_scale=scale,
+                  rel_bias=rb, window=window, softcap=softcap)
+        if kv_range is not None:
+            kw["kv_range"] = kv_range
+        o, lse = oracle.attention(q, k, v, **kw)
+        lo, hi = kv_range if kv_range is not None else (0, Sk)
+        for b in range(B):
+            kl = seqused[b]
+            for h in range(Hq):
+                kh = h // (Hq // Hkv)
+                for i in range(Sq):
+                    e = {}
+                    for j in range(max(lo, 0), min(hi, kl)):
+                        d = i + kl - Sq - j
+                        if (causal and d < 0) or (left >= 0 and d > left) or \
+                                (right >= 0 and -d > right):
+                            continue
+                        s = Decimal(scale) * sum(Decimal(float(q[b, i, h, t])) *
+                                                 Decimal(float(k[b, j, kh, t])) for t in range(D))
+                        if softcap > 0:
+                            s = cap * _dtanh(s / cap)
+                        if 0 <= d < R:
+                            s += Decimal(float(rb[b * Sq + i, h, d]))
+                        e[j] = s.exp()
+                    if not e:
+                        assert lse[b, h, i] == -math.inf and (o[b, i, h] == 0).all()
+                        continue
+                    Z = sum(e.values())
+                    assert lse[b, h, i] == pytest.approx(float(Z.ln()), abs=1e-13)
+                    for t in range(D):
+                        ref = sum(w * Decimal(float(v[b, j, kh, t])) for j, w in e.items()) / Z
+                        assert o[b, i, h, t] == pytest.approx(float(ref), abs=1e-12)
