@@ -520,3 +520,35 @@ def test_dense_modifiers_seqused_and_ranges_high_precision(causal, window, softc
                     for t in range(D):
                         ref = sum(w * Decimal(float(v[b, j, kh, t])) for j, w in e.items()) / Z
                         assert o[b, i, h, t] == pytest.approx(float(ref), abs=1e-12)
+
+
+def test_lse_merge_closed_form_and_degenerate_partials():
+    """The merge of key-range partials against its closed form in decimals:
+    LSE = ln(sum_s e^{LSE_s}), O = sum_s e^{LSE_s} O_s / e^{LSE}.  Partials of
+    magnitude 1000 (e^1000 overflows a double, so the merge must shift by the
+    max), a -inf partial that must carry no weight, and a row that every
+    partial misses (O = 0, LSE = -inf, no NaN)."""
+    getcontext().prec = 50
+    rng = np.random.default_rng(7)
+    S, D = 3, 5
+    lse_parts = np.array([[1000.0, -3.0, 0.5, -math.inf, -math.inf],
+                          [1001.5, -2.0, -math.inf, 2.0, -math.inf],
+                          [999.25, -7.5, 0.25, -math.inf, -math.inf]])
+    o_parts = rng.standard_normal((S, 5, D))
+    co, cl = oracle.lse_combine(o_parts, lse_parts)
+    for r in range(5):
+        live = [s for s in range(S) if lse_parts[s, r] != -math.inf]
+        if not live:
+            assert cl[r] == -math.inf and (co[r] == 0).all()
+            continue
+        w = {s: Decimal(float(lse_parts[s, r])).exp() for s in live}
+        Z = sum(w.values())
+        assert cl[r] == pytest.approx(float(Z.ln()), abs=1e-12)
+        for t in range(D):
+            ref = sum(w[s] * Decimal(float(o_parts[s, r, t])) for s in live) / Z
+            # at |LSE| ~ 1000 one ulp of a double is 1.1e-13, and the weights
+            # exp(LSE_s - LSE) inherit it as a relative error
+            assert co[r, t] == pytest.approx(float(ref), abs=1e-12)
+    # a single live partial passes through unchanged
+    assert cl[3] == 2.0 and (co[3] == o_parts[1, 3]).all()
+    assert np.isfinite(co).all()
