@@ -131,30 +131,47 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(int(stream))
 
 
-def _dtype(q: torch.Tensor) -> int:
+def _dtype(q: torch.Tensor, name: str = "q") -> int:
     if q.dtype not in _DTYPES:
-        raise TypeError(f"q must be bf16 or fp16, got {q.dtype}")
+        raise TypeError(f"{name} must be bf16 or fp16, got {q.dtype}")
     return _DTYPES[q.dtype]
 
 
-def _need_cuda(*ts):
-    for t in ts:
-        if t is not None:
-            if not t.is_cuda:
-                raise ValueError("all tensors must be CUDA tensors")
-            if not t.is_contiguous():
-                raise ValueError("all tensors must be contiguous")
+def _need_args(q, items):
+    """One pass over a call's tensors.  Each (tensor, elements, dtype, name)
+    must hold exactly `elements` elements (the library sees only pointers, so
+    a smaller buffer would be read or written out of bounds on the device),
+    lie on q's device, be contiguous and have `dtype`; None for elements or
+    dtype skips that check.  q's device must be a CUDA device and the current
+    one, since the library launches on the current device."""
+    dev = q.get_device()
+    for t, n, dt, name in items:
+        if t is None:
+            continue
+        if n is not None and t.numel() != n:
+            raise ValueError(f"{name} holds {t.numel()} elements; this call needs {n}")
+        if t.get_device() != dev:
+            raise ValueError(f"{name} is on {t.device}, not on {q.device}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if dt is not None and t.dtype != dt:
+            raise TypeError(f"{name} must be {dt}, got {t.dtype}")
+    if dev < 0:
+        raise ValueError("all tensors must be CUDA tensors")
+    if dev != torch.cuda.current_device():
+        raise ValueError(f"the tensors are on cuda:{dev} but the current device is "
+                         f"cuda:{torch.cuda.current_device()}")
 
 
-def _same_dtype(q, *ts):
-    for t in ts:
-        if t is not None and t.dtype != q.dtype:
-            raise TypeError("q, k, v, out and rel_bias must share one dtype")
+def _dense_shapes(q, k, v):
+    qs, ks = q.shape, k.shape
+    if len(qs) != 4 or len(ks) != 4 or ks[0] != qs[0] or ks[3] != qs[3] or v.shape != ks:
+        raise ValueError("q [B,Sq,Hq,D] and k, v [B,Sk,Hkv,D] shapes disagree")
 
 
-def _int32(t, name):
-    if t is not None and t.dtype != torch.int32:
-        raise TypeError(f"{name} must be int32")
+def _qkv(q, k, v):
+    t = q.dtype
+    return (q, None, t, "q"), (k, None, t, "k"), (v, None, t, "v")
 
 
 def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
@@ -169,18 +186,19 @@ def fa_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
 
     ``window=(left, right)`` and ``softcap`` are the fa_mods modifiers."""
     lib = load_library()
+    _dtype(q)
+    _dense_shapes(q, k, v)
     B, Sq, Hq, D = q.shape
     _, Sk, Hkv, _ = k.shape
-    if k.shape[0] != B or v.shape != k.shape or k.shape[3] != D:
-        raise ValueError("q/k/v shapes disagree")
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
-    _need_cuda(q, k, v, out, lse, seqused_k, rel_bias)
-    _same_dtype(q, k, v, out, rel_bias)
-    _int32(seqused_k, "seqused_k")
     R = 0 if rel_bias is None else int(rel_bias.shape[-1])
+    _need_args(q, _qkv(q, k, v) + (
+        (out, q.numel(), q.dtype, "out"), (lse, B * Hq * Sq, torch.float32, "lse"),
+        (seqused_k, B, torch.int32, "seqused_k"),
+        (rel_bias, B * Sq * Hq * R, q.dtype, "rel_bias")))
     m = _mods(window, softcap)
     _check(lib.fa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq,
                          Sk, Hq, Hkv, D, _dtype(q), int(bool(causal)),
@@ -202,6 +220,9 @@ def fa_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     """Varlen forward: q [total_q,Hq,D], k/v [total_k,Hkv,D] ->
     (out [total_q,Hq,D], lse [Hq,total_q])."""
     lib = load_library()
+    _dtype(q)
+    if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape or k.shape[2] != q.shape[2]:
+        raise ValueError("q [total_q,Hq,D] and k, v [total_k,Hkv,D] shapes disagree")
     total_q, Hq, D = q.shape
     total_k, Hkv, _ = k.shape
     B = int(cu_seqlens_q.shape[0]) - 1
@@ -209,12 +230,13 @@ def fa_fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
-    _need_cuda(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, seqused_k, rel_bias)
-    _same_dtype(q, k, v, out, rel_bias)
-    for t, n in ((cu_seqlens_q, "cu_seqlens_q"), (cu_seqlens_k, "cu_seqlens_k"),
-                 (seqused_k, "seqused_k")):
-        _int32(t, n)
     R = 0 if rel_bias is None else int(rel_bias.shape[-1])
+    _need_args(q, _qkv(q, k, v) + (
+        (out, q.numel(), q.dtype, "out"), (lse, Hq * total_q, torch.float32, "lse"),
+        (cu_seqlens_q, B + 1, torch.int32, "cu_seqlens_q"),
+        (cu_seqlens_k, B + 1, torch.int32, "cu_seqlens_k"),
+        (seqused_k, B, torch.int32, "seqused_k"),
+        (rel_bias, total_q * Hq * R, q.dtype, "rel_bias")))
     m = _mods(window, softcap)
     _check(lib.fa_fwd_varlen_ex(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens_q),
@@ -245,6 +267,8 @@ def fa_fwd_splitkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
                    stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Split-KV dense forward (decode); returns (out, lse [B,Hq,Sq])."""
     lib = load_library()
+    _dtype(q)
+    _dense_shapes(q, k, v)
     B, Sq, Hq, D = q.shape
     _, Sk, Hkv, _ = k.shape
     if out is None:
@@ -258,10 +282,11 @@ def fa_fwd_splitkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
     need = splitkv_workspace_bytes(B, Sq, Hq, D, ns)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    _need_cuda(q, k, v, out, lse, seqused_k, rel_bias, workspace)
-    _same_dtype(q, k, v, out, rel_bias)
-    _int32(seqused_k, "seqused_k")
     R = 0 if rel_bias is None else int(rel_bias.shape[-1])
+    _need_args(q, _qkv(q, k, v) + (
+        (out, q.numel(), q.dtype, "out"), (lse, B * Hq * Sq, torch.float32, "lse"),
+        (seqused_k, B, torch.int32, "seqused_k"),
+        (rel_bias, B * Sq * Hq * R, q.dtype, "rel_bias"), (workspace, None, None, "workspace")))
     m = _mods(window, softcap)
     _check(lib.fa_fwd_splitkv_ex(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq, Sk, Hq, Hkv,
@@ -288,6 +313,8 @@ def fa_fwd_shard_partial(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
     each sequence after the shard).  Returns (o_part [B*Sq*Hq, D] fp32,
     lse_part [B*Sq*Hq] fp32), packed (token, head) rows."""
     lib = load_library()
+    _dtype(q)
+    _dense_shapes(q, k, v)
     B, Sq, Hq, D = q.shape
     _, Sk, Hkv, _ = k.shape
     rows = B * Sq * Hq
@@ -302,14 +329,11 @@ def fa_fwd_shard_partial(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
     if workspace is None and ns > 1:
         workspace = torch.empty(max(splitkv_workspace_bytes(B, Sq, Hq, D, ns), 16),
                                 dtype=torch.uint8, device=q.device)
-    _need_cuda(q, k, v, o_part, lse_part, seqused_k, k_after, rel_bias, workspace)
-    _same_dtype(q, k, v, rel_bias)
-    for t, n in ((o_part, "o_part"), (lse_part, "lse_part")):
-        if t.dtype != torch.float32 or not t.is_contiguous():
-            raise TypeError(f"{n} must be a contiguous float32 tensor")
-    _int32(seqused_k, "seqused_k")
-    _int32(k_after, "k_after")
     R = 0 if rel_bias is None else int(rel_bias.shape[-1])
+    _need_args(q, _qkv(q, k, v) + (
+        (o_part, rows * D, torch.float32, "o_part"), (lse_part, rows, torch.float32, "lse_part"),
+        (seqused_k, B, torch.int32, "seqused_k"), (k_after, B, torch.int32, "k_after"),
+        (rel_bias, B * Sq * Hq * R, q.dtype, "rel_bias"), (workspace, None, None, "workspace")))
     m = _mods(window, softcap)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.fa_fwd_shard_partial(
@@ -335,10 +359,10 @@ def fa_combine_partials(o_parts: torch.Tensor, lse_parts: torch.Tensor, B: int, 
         out = torch.empty((B, Sq, Hq, D), dtype=dtype, device=o_parts.device)
     if lse is None:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=o_parts.device)
-    _need_cuda(o_parts, lse_parts, out, lse)
-    for t, nm in ((o_parts, "o_parts"), (lse_parts, "lse_parts")):
-        if t.dtype != torch.float32 or not t.is_contiguous():
-            raise TypeError(f"{nm} must be a contiguous float32 tensor")
+    _dtype(out, "out")
+    _need_args(o_parts, (
+        (o_parts, None, torch.float32, "o_parts"), (lse_parts, None, torch.float32, "lse_parts"),
+        (out, rows * D, out.dtype, "out"), (lse, rows, torch.float32, "lse")))
     _check(lib.fa_combine_partials(_ptr(o_parts), _ptr(lse_parts), n, B, Sq, Hq, D,
                                    _dtype(out), _ptr(out), _ptr(lse), _stream(stream)))
     return out, lse
@@ -356,16 +380,19 @@ def fa_fwd_splitkv_static(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
     scratch (no workspace); for callers that must not allocate device memory.
     Pass ``out`` and ``lse`` to keep this call free of allocations too."""
     lib = load_library()
+    _dtype(q)
+    _dense_shapes(q, k, v)
     B, Sq, Hq, D = q.shape
     _, Sk, Hkv, _ = k.shape
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
-    _need_cuda(q, k, v, out, lse, seqused_k, rel_bias)
-    _same_dtype(q, k, v, out, rel_bias)
-    _int32(seqused_k, "seqused_k")
     R = 0 if rel_bias is None else int(rel_bias.shape[-1])
+    _need_args(q, _qkv(q, k, v) + (
+        (out, q.numel(), q.dtype, "out"), (lse, B * Hq * Sq, torch.float32, "lse"),
+        (seqused_k, B, torch.int32, "seqused_k"),
+        (rel_bias, B * Sq * Hq * R, q.dtype, "rel_bias")))
     _check(lib.fa_fwd_splitkv_static(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq, Sk, Hq, Hkv,
         D, _dtype(q), int(bool(causal)), float(softmax_scale or 0.0),

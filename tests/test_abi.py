@@ -160,3 +160,86 @@ def test_default_splits_properties(lib):
         bn = 64 if D > 128 else 128
         assert 1 <= ns <= 256
         assert ns <= max(1, -(-Sk // (2 * bn)))  # every split holds at least two key tiles
+
+
+# ---------------------------------------------------------------------------
+# the Python binding's own checks (CPU tensors: every check below fires before
+# anything reaches the library, and a well-formed call on CPU tensors is an
+# error, never a CPU computation)
+# ---------------------------------------------------------------------------
+import torch  # noqa: E402
+
+BF = torch.bfloat16
+
+
+def _dense(B=2, Sq=5, Sk=7, Hq=4, Hkv=2, D=64, dtype=BF):
+    return (torch.zeros(B, Sq, Hq, D, dtype=dtype), torch.zeros(B, Sk, Hkv, D, dtype=dtype),
+            torch.zeros(B, Sk, Hkv, D, dtype=dtype))
+
+
+def _raises(exc, match, fn, *a, **kw):
+    with pytest.raises(exc, match=match):
+        fn(*a, **kw)
+
+
+@pytest.mark.parametrize("call", ["fa_fwd", "fa_fwd_splitkv", "fa_fwd_splitkv_static"])
+def test_binding_rejects_buffers_of_the_wrong_extent(lib, call):
+    fn = getattr(fa, call)
+    kw = {"num_splits": 2} if call != "fa_fwd" else {}
+    q, k, v = _dense()
+    _raises(ValueError, "out holds", fn, q, k, v, out=torch.zeros(2, 5, 4, 63, dtype=BF), **kw)
+    _raises(ValueError, "lse holds", fn, q, k, v, lse=torch.zeros(2, 4, 4), **kw)
+    _raises(TypeError, "lse must be", fn, q, k, v, lse=torch.zeros(2, 4, 5, dtype=BF), **kw)
+    _raises(ValueError, "seqused_k holds", fn, q, k, v,
+            seqused_k=torch.zeros(3, dtype=torch.int32), **kw)
+    _raises(TypeError, "seqused_k must be", fn, q, k, v,
+            seqused_k=torch.zeros(2, dtype=torch.int64), **kw)
+    # rel_bias covers every (token, head): [B*Sq, Hq, R] or [B, Sq, Hq, R]
+    _raises(ValueError, "rel_bias holds", fn, q, k, v,
+            rel_bias=torch.zeros(2 * 5, 3, 128, dtype=BF), **kw)
+    _raises(TypeError, "rel_bias must be", fn, q, k, v,
+            rel_bias=torch.zeros(2, 5, 4, 128, dtype=torch.float16), **kw)
+    _raises(ValueError, "shapes disagree", fn, q, k, v[:, :6].contiguous(), **kw)
+    _raises(ValueError, "shapes disagree", fn, q, k[..., :32].contiguous(),
+            v[..., :32].contiguous(), **kw)
+    _raises(TypeError, "k must be", fn, q, k.half(), v, **kw)
+    _raises(ValueError, "contiguous", fn, q, k, v, out=torch.zeros(2, 4, 5, 64, dtype=BF)
+            .transpose(1, 2), **kw)
+    # everything well formed, but on the CPU: an error, not a fallback
+    _raises(ValueError, "CUDA tensors", fn, q, k, v,
+            rel_bias=torch.zeros(2, 5, 4, 128, dtype=BF),
+            seqused_k=torch.full((2,), 7, dtype=torch.int32), **kw)
+
+
+def test_binding_varlen_extents(lib):
+    q = torch.zeros(9, 4, 64, dtype=BF)
+    k = torch.zeros(11, 2, 64, dtype=BF)
+    cu_q = torch.tensor([0, 4, 9], dtype=torch.int32)
+    cu_k = torch.tensor([0, 5, 11], dtype=torch.int32)
+    f = fa.fa_fwd_varlen
+    _raises(ValueError, "cu_seqlens_k holds", f, q, k, k, cu_q, cu_k[:2], 5, 6)
+    _raises(TypeError, "cu_seqlens_q must be", f, q, k, k, cu_q.long(), cu_k, 5, 6)
+    _raises(ValueError, "lse holds", f, q, k, k, cu_q, cu_k, 5, 6, lse=torch.zeros(4, 8))
+    _raises(ValueError, "rel_bias holds", f, q, k, k, cu_q, cu_k, 5, 6,
+            rel_bias=torch.zeros(8, 4, 128, dtype=BF))
+    _raises(ValueError, "shapes disagree", f, q, k, k[:10].contiguous(), cu_q, cu_k, 5, 6)
+    _raises(ValueError, "shapes disagree", f, q.view(9, 4, 64, 1), k, k, cu_q, cu_k, 5, 6)
+    _raises(ValueError, "CUDA tensors", f, q, k, k, cu_q, cu_k, 5, 6,
+            rel_bias=torch.zeros(9, 4, 128, dtype=BF))
+
+
+def test_binding_shard_partial_and_combine_extents(lib):
+    q, k, v = _dense()
+    f = fa.fa_fwd_shard_partial
+    _raises(ValueError, "k_after holds", f, q, k, v, k_after=torch.zeros(1, dtype=torch.int32))
+    _raises(ValueError, "o_part holds", f, q, k, v, o_part=torch.zeros(40, 63))
+    _raises(TypeError, "lse_part must be", f, q, k, v, lse_part=torch.zeros(40, dtype=BF))
+    _raises(ValueError, "CUDA tensors", f, q, k, v, k_after=torch.zeros(2, dtype=torch.int32))
+    o_parts, l_parts = torch.zeros(3, 40, 64), torch.zeros(3, 40)
+    c = fa.fa_combine_partials
+    _raises(ValueError, "out holds", c, o_parts, l_parts, 2, 5, 4,
+            out=torch.zeros(2, 5, 4, 32, dtype=BF))
+    _raises(TypeError, "lse must be", c, o_parts, l_parts, 2, 5, 4,
+            lse=torch.zeros(2, 4, 5, dtype=BF))
+    _raises(TypeError, "bf16 or fp16", c, o_parts, l_parts, 2, 5, 4, dtype=torch.float32)
+    _raises(ValueError, "CUDA tensors", c, o_parts, l_parts, 2, 5, 4)
