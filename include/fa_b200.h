@@ -40,6 +40,13 @@
  *     head h reads K/V head h / (Hq / Hkv).
  *   - q, k, v, out and rel_bias must be 16-byte aligned and contiguous in the
  *     documented layout.  cu_seqlens and seqused_k are device int32 arrays.
+ *   - The library receives pointers and sizes only, so it cannot check that
+ *     a buffer holds the elements its layout implies for the sizes passed
+ *     (out and q: B*Sq*Hq*D, or total_q*Hq*D; lse: B*Hq*Sq, or Hq*total_q;
+ *     rel_bias: B*Sq*Hq*rel_extent, or total_q*Hq*rel_extent; seqused_k: B;
+ *     cu_seqlens: B+1).  A smaller buffer is read or written out of bounds
+ *     on the device.  The Python binding checks these extents before every
+ *     call.
  *   - softmax_scale <= 0 selects 1 / sqrt(D).
  *   - A query row with no admissible key gets O = 0 and LSE = -inf.
  *   - K/V rows that a call reads but masks (beyond seqused_k, or the padding
