@@ -129,21 +129,28 @@ class ClockSampler:
             self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
             self.ok = True
+            self._read()  # first calls resolve the NVML entry points: keep them out of the region
         except Exception:
             self.ok = False
         self._stop = threading.Event()
         self._t = None
 
-    def _run(self):
+    def _read(self):
+        """(SM clock in MHz, active clock-event reason bits)."""
         nv = self.nv
+        mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except AttributeError:
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        return mhz, int(r)
+
+    def _run(self):
         while not self._stop.is_set():
             try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
-                try:
-                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                except AttributeError:
-                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
-                self.reasons |= int(r)
+                mhz, r = self._read()
+                self.samples.append(mhz)
+                self.reasons |= r
             except Exception:
                 pass
             time.sleep(self.period)

@@ -89,3 +89,36 @@ class _Null:
 
     def __exit__(self, *a):
         return False
+
+
+def test_clock_sampler_with_a_fake_nvml(monkeypatch):
+    """The sampler reads the SM clock and ORs the clock-event reasons while the
+    region runs; `gpu_idle` is not reported; an NVML without the newer reasons
+    call falls back to the older one."""
+    import sys
+    import time
+    import types
+    bench = _bench()
+    state = {"calls": 0}
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=0,
+        nvmlInit=lambda: None,
+        nvmlDeviceGetHandleByIndex=lambda i: ("h", i),
+        nvmlDeviceGetMaxClockInfo=lambda h, c: 1965,
+        nvmlDeviceGetClockInfo=lambda h, c: 1965 if state["calls"] % 2 else 1900,
+    )
+
+    def reasons(h):
+        state["calls"] += 1
+        return 0x1 | (0x4 if state["calls"] > 3 else 0)
+
+    fake.nvmlDeviceGetCurrentClocksThrottleReasons = reasons  # older NVML only
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    s = bench.ClockSampler(0, period_s=0.001)
+    assert s.ok and s.max_mhz == 1965 and not s.samples
+    with s:
+        time.sleep(0.05)
+    out = s.summary()
+    assert out["samples"] >= 3 and out["sm_max_mhz"] == 1965
+    assert out["sm_mhz"] in (1900, 1932.5, 1965)
+    assert out["reasons"] == ["sw_power_cap"]
