@@ -13,7 +13,6 @@ already 0.0156, so the exactly rounded result itself would exceed a bare
 1e-2 (rows that see a handful of keys under a causal mask reach such |O|);
 for |O| well below 1 the added term is negligible.
 """
-import math
 
 import numpy as np
 import torch

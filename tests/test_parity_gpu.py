@@ -5,7 +5,6 @@ compares element by element (tests/parity_util.py states the gates).  Sizes
 span several tiles and a ragged tail; the full-size workloads are checked on
 sampled rows, which the oracle computes one by one exactly.
 """
-import math
 
 import numpy as np
 import pytest

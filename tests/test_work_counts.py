@@ -9,7 +9,6 @@ count of admitted (row, key) pairs written out from the distance rule.
 import itertools
 
 import pytest
-import torch
 
 import fa_inputs
 
