@@ -243,3 +243,41 @@ def test_binding_shard_partial_and_combine_extents(lib):
             lse=torch.zeros(2, 4, 5, dtype=BF))
     _raises(TypeError, "bf16 or fp16", c, o_parts, l_parts, 2, 5, 4, dtype=torch.float32)
     _raises(ValueError, "CUDA tensors", c, o_parts, l_parts, 2, 5, 4)
+
+
+def _kind_of_c(param: str) -> str:
+    """Kind of one C parameter as the header spells it."""
+    p = " ".join(param.split())
+    if "*" in p:
+        return "ptr"
+    base = " ".join(w for w in p.split()[:-1] if w != "const")
+    # size_t and unsigned long long are both 64-bit unsigned here (LP64),
+    # and ctypes makes c_size_t and c_ulonglong one type
+    return {"int": "i32", "fa_dtype": "i32", "fa_status": "i32", "float": "f32",
+            "size_t": "u64", "unsigned long long": "u64"}[base]
+
+
+def _kind_of_ctypes(t) -> str:
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or isinstance(t, type(ctypes.POINTER(ctypes.c_int))):
+        return "ptr"
+    assert ctypes.sizeof(t) in (4, 8)
+    return {ctypes.c_int: "i32", ctypes.c_float: "f32", ctypes.c_size_t: "u64",
+            ctypes.c_ulonglong: "u64"}[t]
+
+
+def test_binding_signatures_match_the_header(lib):
+    """Every entry point the header declares has ctypes argtypes in the
+    binding with the same number of parameters of the same kinds, so that a
+    change on one side cannot silently shift the arguments of the other."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    protos = {m.group(1): m.group(2) for m in
+              re.finditer(r"\b(fa_\w+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S)}
+    assert len(protos) >= 16
+    for name, params in protos.items():
+        params = " ".join(params.split())
+        want = [] if params in ("", "void") else [_kind_of_c(x) for x in params.split(",")]
+        got = getattr(lib, name).argtypes
+        assert got is not None, f"{name}: the binding declares no argtypes"
+        assert [_kind_of_ctypes(t) for t in got] == want, name
