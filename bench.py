@@ -4,12 +4,14 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 One step is one forward over one batch of the main workload (default: the
-varlen causal GQA 32/8 D=128 workload with a 256-wide relative bias, 4
-sequences of seeded lengths in [512, 4096]).  Rank 0 prints ONE JSON line with
+largest single-GPU configuration, dense non-causal MHA B=1 S=20480 H=56 D=128
+bf16, the long video-DiT validation shape).  Rank 0 prints ONE JSON line with
 the throughput in TFLOP/s (4 * q_len * k_len * D * Hq per sequence, halved for
 causal), the roofline of the kernel, the CPU oracle baseline, an end-to-end
 figure through host buffers, the SM clocks seen while timing, and the other
-workloads measured the same way ("workloads").
+workloads measured the same way ("workloads"; among them the varlen causal
+GQA 32/8 D=128 workload with a 256-wide relative bias, and fp16 twins of two
+bf16 workloads).
 
 Multi-GPU (launched by torchrun): every rank runs its own copy of the workload
 (independent problems, no data-path collective: weak scaling); the time is the
@@ -35,9 +37,13 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "attention fwd TFLOP/s & % of BF16 tensor peak; split-KV decode HBM GB/s"
-MAIN = "varlen_gqa_bias"
-EXTRAS = ["dense_257", "video_dit_20480", "encoder_d256_seqused", "decode_splitkv", "dense_d64",
+MAIN = "video_dit_20480"
+EXTRAS = ["varlen_gqa_bias", "dense_257", "encoder_d256_seqused", "decode_splitkv", "dense_d64",
           "local_window_softcap", "tabpfn_d16", "vision_d72"]
+# the same shapes in fp16: a bf16 / fp16 pair per shape ("FlashAttention-4
+# backend for Blackwell #1235", Benchmarking, reports a bf16 slow-down on sm_100)
+FP16_TWINS = ["video_dit_20480", "dense_d64"]
+L2_BYTES = 126 << 20  # B200; the device's own figure replaces it where CUDA is up
 DESCR = {
     "dense_257": "dense non-causal MHA B=1 S=257 H=8 D=128 bf16",
     "varlen_gqa_bias": "varlen causal GQA 32/8 D=128, 4 seqs U[512,4096] (seeded), rel_bias R=256 bf16",
@@ -177,17 +183,32 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # workloads on the device
 # ---------------------------------------------------------------------------
-BIG = {"video_dit_20480", "decode_splitkv"}
+BIG = {"decode_splitkv"}
 
 
 DECODE_SK = 131072
 
 
-def build_problem(name: str, device):
+def build_problem(name: str, device, dtype=None):
+    import torch
     import fa_inputs
+    dtype = dtype or torch.bfloat16
     if name in BIG:
-        return fa_inputs.make(name, device=device, decode_sk=DECODE_SK)
-    return fa_inputs.make(name).to(device)
+        return fa_inputs.make(name, dtype=dtype, device=device, decode_sk=DECODE_SK)
+    return fa_inputs.make(name, dtype=dtype).to(device)
+
+
+def workload_config(name: str, p, world: int, l2_bytes: int = L2_BYTES) -> dict:
+    """The `config` object of the JSON line: the workload and how it is timed.
+    Both arms print the same one for the same workload."""
+    small = p.hbm_bytes() < 2 * l2_bytes
+    return {"workload": f"{name}: {DESCR[name]}", "global_batch": p.B * world,
+            "seq_len": p.max_seqlen_q,
+            "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU",
+            "l2": (f"{p.hbm_bytes() / 1e6:.0f} MB touched per step < 2 x L2: a buffer of 4 x L2 "
+                   "is overwritten before every step, outside its events; time = per-step "
+                   "event mean" if small else
+                   f"inputs larger than L2 ({p.hbm_bytes() / 1e6:.0f} MB per step), no flush")}
 
 
 class Runner:
@@ -571,10 +592,11 @@ def main():
     # ---- the other workloads, same protocol (rank 0 reports its own)
     extras = {}
     if not a.no_extras:
-        for name in EXTRAS:
-            if name == a.workload:
-                continue
-            q = build_problem(name, dev)
+        runs = [(n, False) for n in EXTRAS if n != a.workload]
+        runs += [(n, True) for n in FP16_TWINS]
+        for name, twin in runs:
+            key = name + "_fp16" if twin else name
+            q = build_problem(name, dev, torch.float16 if twin else None)
             r = Runner(q, a.splits)
             k_steps = max(5, min(a.steps, 30))
             small = q.hbm_bytes() < 2 * l2_bytes
@@ -587,15 +609,16 @@ def main():
                 tt = pm * k_steps  # the flush between steps is not the workload's time
             tt = max_over_ranks(tt, dist_on)
             v, u = workload_value(q, tt / k_steps)
-            rf = roofline(q, pm, peaks, profiled_traffic(name))
-            extras[name] = {"workload": DESCR[name], "value": round(world * v, 3), "unit": u,
+            rf = roofline(q, pm, peaks, None if twin else profiled_traffic(name))
+            extras[key] = {"workload": DESCR[name] + (" (fp16 twin)" if twin else ""),
+                           "value": round(world * v, 3), "unit": u,
                             "ms_per_step": round(tt / k_steps, 4), "frac_of_peak": rf["frac"],
                             "roofline": rf, "gpu_launches_per_step": r.launches,
                             "sm_mhz": ck.get("sm_mhz"),
                             "l2": ("flushed before every step (inputs fit in L2), per-step events"
                                    if small else "inputs larger than L2, no flush")}
             if q.splitkv:
-                extras[name]["num_splits"] = r.ns
+                extras[key]["num_splits"] = r.ns
             del q, r
             torch.cuda.empty_cache()
 
@@ -618,14 +641,8 @@ def main():
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) inputs of the workload's shape)",
-        "config": {"workload": f"{a.workload}: {DESCR[a.workload]}",
-                   "global_batch": p.B * world, "seq_len": p.max_seqlen_q,
-                   "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU",
-                   "l2": (f"{p.hbm_bytes() / 1e6:.0f} MB touched per step < 2 x L2: a "
-                          f"{flush_buf.numel() >> 20} MiB buffer is overwritten before every step, "
-                          "outside its events; time = per-step event mean" if main_small else
-                          f"inputs larger than L2 ({p.hbm_bytes() / 1e6:.0f} MB per step), no flush"),
-                   "pct_of_bf16_peak": round(100 * roof["frac"], 2) if roof["bound"] == "tensor" else None},
+        "config": workload_config(a.workload, p, world, l2_bytes),
+        "pct_of_bf16_peak": round(100 * roof["frac"], 2) if roof["bound"] == "tensor" else None,
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -675,8 +692,7 @@ def run_reference(a, world):
             "ms_per_step": round(1e3 * dt / a.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded N(0,1) inputs of the workload's shape)",
-            "config": {"workload": f"{name}: {DESCR[name]}", "global_batch": p.B,
-                       "seq_len": p.max_seqlen_q, "parallelism": "CPU oracle"},
+            "config": workload_config(name, p, world),
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s",
                              "cores": oracle.num_threads(), "kind": "oracle",
                              "sample": f"{n0} random rows per step of {name}, fp64 C/OpenMP"},

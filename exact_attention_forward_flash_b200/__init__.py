@@ -99,6 +99,8 @@ def load_library(path: Optional[str] = None):
     lib.fa_combine_partials.restype = i32
     lib.fa_watchdog_selftest.argtypes = [ctypes.c_ulonglong, P]
     lib.fa_watchdog_selftest.restype = i32
+    lib.fa_selftest_exp2_fma.argtypes = [P, P, ctypes.c_longlong, P]
+    lib.fa_selftest_exp2_fma.restype = i32
     lib.fa_check_device_error.argtypes = [ctypes.POINTER(i32), i32]
     lib.fa_check_device_error.restype = i32
     lib.fa_status_string.argtypes = [i32]
@@ -400,13 +402,29 @@ def fa_fwd_splitkv_static(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *,
     return out, lse
 
 
+FA_ERR_DEVICE_TIMEOUT, FA_ERR_DEVICE_INPUT = 5, 6
+DEVICE_TIMEOUT, DEVICE_INPUT = 1, 2   # bits of the device error word
+
+
 def check_device_error(clear: bool = True) -> int:
-    """Synchronise and return the kernels' watchdog word (0 = no timeout)."""
+    """Synchronise and return the kernels' device error word: 0 = none, bit 1
+    (DEVICE_TIMEOUT) a wait gave up, bit 2 (DEVICE_INPUT) a sequence broke
+    the cu_seqlens / seqused_k contract and was skipped."""
     code = ctypes.c_int(0)
     st = load_library().fa_check_device_error(ctypes.byref(code), int(clear))
-    if st not in (FA_OK, 5):
+    if st not in (FA_OK, FA_ERR_DEVICE_TIMEOUT, FA_ERR_DEVICE_INPUT):
         _check(st)
     return int(code.value)
+
+
+def selftest_exp2_fma(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """2^x through the softmax's FMA-pipe exponential (a device self-test of
+    that routine); x is a contiguous float32 CUDA tensor."""
+    lib = load_library()
+    y = torch.empty_like(x)
+    _need_args(x, ((x, None, torch.float32, "x"), (y, x.numel(), torch.float32, "y")))
+    _check(lib.fa_selftest_exp2_fma(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
+    return y
 
 
 def watchdog_selftest(timeout_s: float = 0.05, stream=None) -> None:

@@ -1,9 +1,15 @@
 """Build the CUDA library in-tree: csrc/*.cu -> libfa_b200.so (sm_100a).
 
-    python -m exact_attention_forward_flash_b200.build [--force]
+    python -m exact_attention_forward_flash_b200.build [--force] [-v]
+
+Each translation unit (the C ABI in fa_api.cu, one fa_kern_w<W>.cu per kernel
+width) compiles to an object file in parallel; nvcc then links the shared
+library.  The objects go to a temporary folder that is removed afterwards.
 """
 from __future__ import annotations
 
+import concurrent.futures
+import tempfile
 import glob
 import os
 import shutil
@@ -48,16 +54,29 @@ def needs_build() -> bool:
     return any(os.path.getmtime(f) > t for f in _deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, jobs: int = 0) -> str:
     """Compile the library unless it is up to date; returns its path."""
     if not force and not needs_build():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *_sources()]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-        print(" ".join(cmd), flush=True)
-    subprocess.check_call(cmd)
+    nvcc = _nvcc()
+    compile_flags = [f for f in NVCC_FLAGS if f != "-shared"]
+    srcs = _sources()
+    jobs = jobs or min(len(srcs), os.cpu_count() or 1)
+    with tempfile.TemporaryDirectory(prefix="fa_b200_build_") as tmpdir:
+        def compile_one(src):
+            obj = os.path.join(tmpdir, os.path.basename(src) + ".o")
+            cmd = [nvcc, *compile_flags, "-I", INCLUDE, "-I", CSRC, "-c", "-o", obj, src]
+            if verbose:
+                cmd.insert(1, "-Xptxas=-v")
+                print(" ".join(cmd), flush=True)
+            subprocess.check_call(cmd)
+            return obj
+
+        with concurrent.futures.ThreadPoolExecutor(max_workers=jobs) as ex:
+            objs = list(ex.map(compile_one, srcs))
+        tmp = LIB + f".tmp{os.getpid()}"
+        subprocess.check_call([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
+                               "-Xcompiler", "-fPIC", "-o", tmp, *objs])
     os.replace(tmp, LIB)
     return LIB
 

@@ -1,7 +1,9 @@
 // fa_api.cu -- the C ABI of the attention forward library (declared in
 // include/fa_b200.h): argument validation, TMA descriptor encoding, kernel
-// selection and launch.  Nothing here allocates device memory or synchronises
-// a stream (fa_check_device_error excepted, by its contract).
+// selection and launch, the split-KV merge.  The forward kernels themselves
+// are instantiated per width in fa_kern_w<W>.cu.  Nothing here allocates
+// device memory or synchronises a stream (fa_check_device_error excepted, by
+// its contract).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -12,13 +14,18 @@
 #include <mutex>
 
 #include "fa_b200.h"
-#include "fa_fwd_kernel.cuh"
+#include "fa_launch.cuh"
+
+// The library's device error word (one per device): kernels record timeouts
+// and broken input contracts here (see sm100_ptx.cuh); fa_check_device_error
+// reads and clears it.
+static __device__ unsigned g_fa_error;
 
 namespace {
-
-using namespace fab;
-
 thread_local char g_msg[512] = "";
+}  // namespace
+
+namespace fab {
 
 fa_status fail(fa_status s, const char *fmt, ...) {
   va_list ap;
@@ -27,6 +34,61 @@ fa_status fail(fa_status s, const char *fmt, ...) {
   va_end(ap);
   return s;
 }
+
+int num_sms(int dev) {
+  static int cache[kMaxDev] = {0};
+  if (dev < 0 || dev >= kMaxDev) return 148;
+  if (cache[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      v = 148;
+    cache[dev] = v;
+  }
+  return cache[dev];
+}
+
+}  // namespace fab
+
+namespace fab {
+
+// ---------------------------------------------------------------------------
+// watchdog self-test: one thread waits, bounded by timeout_ns, on a fresh
+// mbarrier that nothing ever arrives at, so the wait must give up, record the
+// timeout code in the watchdog word and return (no trap, no endless loop).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(32) fa_watchdog_selftest_kernel(unsigned *err,
+                                                                  unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) (void)mbar_wait(smem_u32(&bar), 0u, err, timeout_ns);
+}
+
+// ---------------------------------------------------------------------------
+// FMA-pipe exponential self-test: y = 2^x through ex2_poly2, the routine the
+// softmax uses for part of its exponentials, element pairs per thread (an odd
+// last element is paired with 0).  Lets a test measure its error on the GPU.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) fa_selftest_exp2_fma_kernel(const float *__restrict__ x,
+                                                                   float *__restrict__ y,
+                                                                   long long n) {
+  const long long i = 2 * ((long long)blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const bool pair = i + 1 < n;
+  float y0, y1;
+  ex2_poly2(x[i], pair ? x[i + 1] : 0.f, y0, y1);
+  y[i] = y0;
+  if (pair) y[i + 1] = y1;
+}
+
+}  // namespace fab
+
+namespace {
+
+using namespace fab;
 
 // ---------------------------------------------------------------------------
 // driver entry point for tensor-map encoding (no link-time libcuda dependency)
@@ -120,74 +182,52 @@ fa_status encode_map(CUtensorMap *tm, const void *base, int D, int H, long long 
 // ---------------------------------------------------------------------------
 // per-device state
 // ---------------------------------------------------------------------------
-constexpr int kMaxDev = 64;
-
-int num_sms(int dev) {
-  static int cache[kMaxDev] = {0};
-  if (dev < 0 || dev >= kMaxDev) return 148;
-  if (cache[dev] == 0) {
-    int v = 0;
-    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
-      v = 148;
-    cache[dev] = v;
+// Device address of a __device__ variable, looked up with `dev` current (the
+// caller passes the current device) and cached per device.
+template <class T>
+fa_status symbol_address(T &sym, int dev, void **cache, std::mutex &mu, void **addr,
+                         const char *what) {
+  if (dev < 0 || dev >= kMaxDev) return fail(FA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == nullptr) {
+    void *ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, sym);
+    if (e != cudaSuccess || ptr == nullptr)
+      return fail(FA_ERR_CUDA, "looking up %s: %s", what, cudaGetErrorString(e));
+    cache[dev] = ptr;
   }
-  return cache[dev];
-}
-
-// kernel variants
-// kernel configurations by (16-bit format: bf16 / fp16, modifiers off / on)
-template <bool H, bool M> using Fwd16 = FwdCfg<16, 128, 2, 1, 3, 0, H, false, M>;
-template <bool H, bool M> using Fwd32 = FwdCfg<32, 128, 2, 1, 3, 0, H, false, M>;
-template <bool H, bool M> using Fwd48 = FwdCfg<48, 128, 2, 1, 3, 0, H, false, M>;
-template <bool H, bool M> using Fwd80 = FwdCfg<80, 128, 2, 1, 3, 0, H, false, M>;
-template <bool H, bool M> using Fwd96 = FwdCfg<96, 128, 2, 1, 3, 0, H, false, M>;
-template <bool H, bool M> using Fwd64 = FwdCfg<64, 128, 2, 1, 3, 0, H, false, M>;
-template <bool H, bool M> using Fwd128 = FwdCfg<128, 128, 2, 1, 3, 0, H, false, M>;
-template <bool H, bool M> using Fwd256 = FwdCfg<256, 64, 1, 2, 3, 2, H, false, M>;
-// one Q tile per CTA with a double-buffered S: each unit runs at the
-// softmax's own rate instead of sharing its SMSPs with a second tile; for
-// problems with fewer two-tile units than SMs (latency-bound calls)
-template <bool H, bool M> using Lat16 = FwdCfg<16, 128, 1, 2, 3, 3, H, false, M>;
-template <bool H, bool M> using Lat32 = FwdCfg<32, 128, 1, 2, 3, 3, H, false, M>;
-template <bool H, bool M> using Lat48 = FwdCfg<48, 128, 1, 2, 3, 3, H, false, M>;
-template <bool H, bool M> using Lat64 = FwdCfg<64, 128, 1, 2, 3, 3, H, false, M>;
-template <bool H, bool M> using Lat80 = FwdCfg<80, 128, 1, 2, 3, 3, H, false, M>;
-template <bool H, bool M> using Lat96 = FwdCfg<96, 128, 1, 2, 3, 3, H, false, M>;
-template <bool H, bool M> using Lat128 = FwdCfg<128, 128, 1, 2, 3, 3, H, false, M>;
-template <bool H, bool M> using Spl16 = FwdCfg<16, 128, 1, 2, 3, 3, H, true, M>;
-template <bool H, bool M> using Spl32 = FwdCfg<32, 128, 1, 2, 3, 3, H, true, M>;
-template <bool H, bool M> using Spl48 = FwdCfg<48, 128, 1, 2, 3, 3, H, true, M>;
-template <bool H, bool M> using Spl80 = FwdCfg<80, 128, 1, 2, 3, 3, H, true, M>;
-template <bool H, bool M> using Spl96 = FwdCfg<96, 128, 1, 2, 3, 3, H, true, M>;
-template <bool H, bool M> using Spl64 = FwdCfg<64, 128, 1, 2, 3, 3, H, true, M>;
-template <bool H, bool M> using Spl128 = FwdCfg<128, 128, 1, 2, 3, 3, H, true, M>;
-template <bool H, bool M> using Spl256 = FwdCfg<256, 64, 1, 2, 2, 2, H, true, M>;
-
-template <class C>
-fa_status launch_fwd(FwdParams &p, int dev, cudaStream_t st) {
-  static bool configured[kMaxDev] = {false};
-  if (dev >= 0 && dev < kMaxDev && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(fa_fwd_kernel<C>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
-    if (e != cudaSuccess)
-      return fail(FA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    configured[dev] = true;
-  }
-  // causal problems with few enough sequences use the compact schedule
-  p.compact = (p.m_major && p.B >= 1 && p.B <= C::kMaxSchedB) ? 1 : 0;
-  const int grid = std::min(p.num_units, num_sms(dev));
-  fa_fwd_kernel<C><<<grid, C::kThreads, C::kSmemBytes, st>>>(p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
+  *addr = cache[dev];
   return FA_OK;
 }
 
-// one of the four variants of a configuration
-template <template <bool, bool> class Cfg>
-fa_status launch_variant(FwdParams &p, int dev, cudaStream_t st, bool half, bool mods) {
-  if (half) return mods ? launch_fwd<Cfg<true, true>>(p, dev, st) : launch_fwd<Cfg<true, false>>(p, dev, st);
-  return mods ? launch_fwd<Cfg<false, true>>(p, dev, st) : launch_fwd<Cfg<false, false>>(p, dev, st);
+fa_status error_word(int dev, unsigned **addr) {
+  static std::mutex mu;
+  static void *cache[kMaxDev] = {nullptr};
+  void *a = nullptr;
+  fa_status s = symbol_address(g_fa_error, dev, cache, mu, &a, "the device error word");
+  *addr = static_cast<unsigned *>(a);
+  return s;
+}
+
+// The current device and its error word.
+fa_status current_device(int *dev, unsigned **err) {
+  if (cudaGetDevice(dev) != cudaSuccess) return fail(FA_ERR_CUDA, "cudaGetDevice failed");
+  return error_word(*dev, err);
+}
+
+// The kernel of width w and kind k.
+fa_status launch_width(int w, Kind k, FwdParams &p, int dev, cudaStream_t st, bool half,
+                       bool mods) {
+  switch (w) {
+    case 16: return launch_w16(k, p, dev, st, half, mods);
+    case 32: return launch_w32(k, p, dev, st, half, mods);
+    case 48: return launch_w48(k, p, dev, st, half, mods);
+    case 64: return launch_w64(k, p, dev, st, half, mods);
+    case 80: return launch_w80(k, p, dev, st, half, mods);
+    case 96: return launch_w96(k, p, dev, st, half, mods);
+    case 128: return launch_w128(k, p, dev, st, half, mods);
+    default: return launch_w256(k, p, dev, st, half, mods);
+  }
 }
 
 // the modifier kernels serve a left window bound or a soft-cap (the plain
@@ -253,8 +293,11 @@ fa_status validate(const Common &c) {
     if (c.R <= 0 || c.R % 128 != 0)
       return fail(FA_ERR_INVALID, "rel_extent (%d) must be a positive multiple of 128", c.R);
     if (!aligned16(c.rel_bias)) return fail(FA_ERR_INVALID, "rel_bias must be 16-byte aligned");
-    const long long tqb = c.varlen ? c.total_q : (long long)c.B * c.Sq;
-    if (tqb * c.Hq * (long long)c.R / 8 >= (1LL << 32))
+    // B * Sq * Hq * rel_extent elements of 2 bytes; the product is taken in
+    // 128 bits (B * Sq alone may reach 2^62 before the token-count rule)
+    const unsigned __int128 tqb =
+        c.varlen ? (unsigned __int128)c.total_q : (unsigned __int128)c.B * (unsigned)c.Sq;
+    if (tqb * (unsigned)c.Hq * (unsigned)c.R * 2u >= ((unsigned __int128)64 << 30))
       return fail(FA_ERR_UNSUPPORTED, "rel_bias larger than 64 GiB");
   }
   if (!std::isfinite(c.scale)) return fail(FA_ERR_INVALID, "softmax_scale must be finite");
@@ -321,7 +364,9 @@ fa_status fill_params(const Common &c, FwdParams &p, int nq, int bn, int num_spl
   while ((1 << p.lgP) < P) ++p.lgP;
   p.n_groups = c.Hq / P;
   p.total_q = (int)tq;
+  p.total_k = (int)tk;
   const int max_q = c.varlen ? c.max_q : c.Sq;
+  p.max_q = max_q;
   const long long rows = (long long)max_q * P;
   p.n_mblk = (int)std::max<long long>(1, (rows + (long long)nq * kBM - 1) / ((long long)nq * kBM));
   p.num_splits = num_splits;
@@ -352,7 +397,8 @@ fa_status run_fwd(const Common &c, cudaStream_t st) {
   const long long tq = c.varlen ? c.total_q : (long long)c.B * c.Sq;
   if (tq == 0 || c.B == 0) return FA_OK;  // nothing to compute
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return fail(FA_ERR_CUDA, "cudaGetDevice failed");
+  unsigned *err = nullptr;
+  if ((s = current_device(&dev, &err)) != FA_OK) return s;
   FwdParams p;
   // width <= 128: two Q tiles per CTA, 128-key tiles; 256: one Q tile, 64-key tiles
   const int w = kernel_width(c.D);
@@ -361,29 +407,14 @@ fa_status run_fwd(const Common &c, cudaStream_t st) {
   if (p.num_units == 0) return FA_OK;
   const bool half = c.dt == FA_FP16;
   const bool mods = uses_mods(p);
+  Kind kind = Kind::kThroughput;
   if (w <= 128 && p.num_units < num_sms(dev)) {
     // fewer two-tile units than SMs: one tile per CTA, twice the units
     if ((s = fill_params(c, p, 1, 128, 1, 0x7fffffff)) != FA_OK) return s;
-    switch (w) {
-      case 16: return launch_variant<Lat16>(p, dev, st, half, mods);
-      case 32: return launch_variant<Lat32>(p, dev, st, half, mods);
-      case 48: return launch_variant<Lat48>(p, dev, st, half, mods);
-      case 64: return launch_variant<Lat64>(p, dev, st, half, mods);
-      case 80: return launch_variant<Lat80>(p, dev, st, half, mods);
-      case 96: return launch_variant<Lat96>(p, dev, st, half, mods);
-      default: return launch_variant<Lat128>(p, dev, st, half, mods);
-    }
+    kind = Kind::kLatency;
   }
-  switch (w) {
-    case 16: return launch_variant<Fwd16>(p, dev, st, half, mods);
-    case 32: return launch_variant<Fwd32>(p, dev, st, half, mods);
-    case 48: return launch_variant<Fwd48>(p, dev, st, half, mods);
-    case 64: return launch_variant<Fwd64>(p, dev, st, half, mods);
-    case 80: return launch_variant<Fwd80>(p, dev, st, half, mods);
-    case 96: return launch_variant<Fwd96>(p, dev, st, half, mods);
-    case 128: return launch_variant<Fwd128>(p, dev, st, half, mods);
-    default: return launch_variant<Fwd256>(p, dev, st, half, mods);
-  }
+  p.err = err;
+  return launch_width(w, kind, p, dev, st, half, mods);
 }
 
 template <int D, bool HALF, bool F32OUT>
@@ -440,6 +471,24 @@ fa_status combine(int D, bool half, bool f32out, const float *o_part, const floa
 
 int splitkv_bn(int D) { return kernel_width(D) == 256 ? 64 : 128; }
 
+// The split count a split-KV call launches and the keys of each split
+// (whole key tiles): num_splits (0 = the default for this device) capped at
+// one split per key tile, then reduced to the splits that the rounded split
+// length actually needs.
+struct SplitPlan {
+  int ns, split_keys;
+};
+
+SplitPlan plan_splits(int B, int Sq, int Sk, int Hq, int Hkv, int D, int num_splits, int n_sms) {
+  const int bn = splitkv_bn(D);
+  int ns = num_splits > 0 ? num_splits : fa_splitkv_default_splits(B, Sq, Sk, Hq, Hkv, D, n_sms);
+  const long long tiles = std::max<long long>(1, ((long long)Sk + bn - 1) / bn);
+  if (ns > tiles) ns = (int)tiles;
+  if (ns < 1) ns = 1;
+  const int split_keys = (int)(((tiles + ns - 1) / ns) * bn);
+  ns = (int)std::max<long long>(1, ((long long)Sk + split_keys - 1) / split_keys);
+  return {ns, split_keys};
+}
 
 // Split-KV forward of a dense problem: the keys are cut into num_splits
 // ranges whose normalised fp32 partials go to the workspace and are merged
@@ -454,15 +503,12 @@ fa_status run_splitkv(const Common &c, int num_splits, void *workspace, size_t w
   const int B = c.B, Sq = c.Sq, Sk = c.Sk, Hq = c.Hq, D = c.D;
   if ((long long)B * Sq == 0) return FA_OK;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return fail(FA_ERR_CUDA, "cudaGetDevice failed");
+  unsigned *err = nullptr;
+  if ((s = current_device(&dev, &err)) != FA_OK) return s;
   if (Sk == 0 && !to_partial) return run_fwd(c, st);  // nothing to split
   const int bn = splitkv_bn(D);
-  int ns = num_splits > 0 ? num_splits
-                          : fa_splitkv_default_splits(B, Sq, Sk, Hq, c.Hkv, D, num_sms(dev));
-  const long long tiles = std::max<long long>(1, ((long long)Sk + bn - 1) / bn);
-  if (ns > tiles) ns = (int)tiles;
-  const int split_keys = (int)(((tiles + ns - 1) / ns) * bn);
-  ns = (int)std::max<long long>(1, ((long long)Sk + split_keys - 1) / split_keys);
+  const SplitPlan sp = plan_splits(B, Sq, Sk, Hq, c.Hkv, D, num_splits, num_sms(dev));
+  const int ns = sp.ns;
   const long long rows = (long long)B * Sq * Hq;
   const bool direct = to_partial && ns == 1;
   if (!direct) {
@@ -473,7 +519,8 @@ fa_status run_splitkv(const Common &c, int num_splits, void *workspace, size_t w
     if (!aligned16(workspace)) return fail(FA_ERR_INVALID, "workspace must be 16-byte aligned");
   }
   FwdParams p;
-  if ((s = fill_params(c, p, 1, bn, ns, split_keys)) != FA_OK) return s;
+  if ((s = fill_params(c, p, 1, bn, ns, sp.split_keys)) != FA_OK) return s;
+  p.err = err;
   if (direct) {
     p.o_part = static_cast<float *>(c.out);
     p.lse_part = c.lse;
@@ -484,17 +531,7 @@ fa_status run_splitkv(const Common &c, int num_splits, void *workspace, size_t w
   // fp32 partial rows hold D * 4 bytes (a multiple of 32): only the base counts
   p.st32 = (reinterpret_cast<uintptr_t>(p.o_part) & 31) == 0 ? 1 : 0;
   const bool half = c.dt == FA_FP16;
-  const bool mods = uses_mods(p);
-  switch (kernel_width(D)) {
-    case 16: s = launch_variant<Spl16>(p, dev, st, half, mods); break;
-    case 32: s = launch_variant<Spl32>(p, dev, st, half, mods); break;
-    case 48: s = launch_variant<Spl48>(p, dev, st, half, mods); break;
-    case 64: s = launch_variant<Spl64>(p, dev, st, half, mods); break;
-    case 80: s = launch_variant<Spl80>(p, dev, st, half, mods); break;
-    case 96: s = launch_variant<Spl96>(p, dev, st, half, mods); break;
-    case 128: s = launch_variant<Spl128>(p, dev, st, half, mods); break;
-    default: s = launch_variant<Spl256>(p, dev, st, half, mods); break;
-  }
+  s = launch_width(kernel_width(D), Kind::kPartial, p, dev, st, half, uses_mods(p));
   if (s != FA_OK || direct) return s;
   return combine(D, half, to_partial, p.o_part, p.lse_part, ns, rows, c.out, c.lse, Hq, Sq, B,
                  st);
@@ -654,7 +691,26 @@ fa_status fa_watchdog_selftest(unsigned long long timeout_ns, void *stream) {
   g_msg[0] = 0;
   if (timeout_ns < 1000000ull || timeout_ns > 1000000000ull)
     return fail(FA_ERR_INVALID, "timeout_ns must be within [1 ms, 1 s]");
-  fab::fa_watchdog_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
+  int dev = 0;
+  unsigned *err = nullptr;
+  fa_status s = current_device(&dev, &err);
+  if (s != FA_OK) return s;
+  fab::fa_watchdog_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(err, timeout_ns);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FA_ERR_CUDA, "self-test launch: %s", cudaGetErrorString(e));
+  return FA_OK;
+}
+
+fa_status fa_selftest_exp2_fma(const float *x, float *y, long long n, void *stream) {
+  g_msg[0] = 0;
+  if (n < 0) return fail(FA_ERR_INVALID, "n must be >= 0");
+  if (n == 0) return FA_OK;
+  if (x == nullptr || y == nullptr) return fail(FA_ERR_INVALID, "x and y must not be NULL");
+  const long long threads = 256, pairs = (n + 1) / 2;
+  const long long blocks = (pairs + threads - 1) / threads;
+  if (blocks > 0x7fffffffLL) return fail(FA_ERR_UNSUPPORTED, "n too large");
+  fab::fa_selftest_exp2_fma_kernel<<<(unsigned)blocks, (unsigned)threads, 0,
+                                     static_cast<cudaStream_t>(stream)>>>(x, y, n);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(FA_ERR_CUDA, "self-test launch: %s", cudaGetErrorString(e));
   return FA_OK;
@@ -664,15 +720,17 @@ fa_status fa_check_device_error(int *code, int clear) {
   unsigned v = 0;
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return fail(FA_ERR_CUDA, "cudaDeviceSynchronize: %s", cudaGetErrorString(e));
-  e = cudaMemcpyFromSymbol(&v, fab::g_fa_error, sizeof(v));
+  e = cudaMemcpyFromSymbol(&v, g_fa_error, sizeof(v));
   if (e != cudaSuccess) return fail(FA_ERR_CUDA, "reading the error word: %s", cudaGetErrorString(e));
   if (code) *code = (int)v;
   if (clear && v) {
     unsigned z = 0;
-    e = cudaMemcpyToSymbol(fab::g_fa_error, &z, sizeof(z));
+    e = cudaMemcpyToSymbol(g_fa_error, &z, sizeof(z));
     if (e != cudaSuccess) return fail(FA_ERR_CUDA, "clearing the error word: %s", cudaGetErrorString(e));
   }
-  return v ? FA_ERR_DEVICE_TIMEOUT : FA_OK;
+  if (v & fab::kErrTimeout) return FA_ERR_DEVICE_TIMEOUT;
+  if (v & fab::kErrInput) return FA_ERR_DEVICE_INPUT;
+  return FA_OK;
 }
 
 }  // extern "C"
@@ -693,18 +751,8 @@ namespace {
 
 fa_status splitkv_scratch_address(int dev, void **addr) {
   static std::mutex mu;
-  static void *cached[kMaxDev] = {nullptr};
-  if (dev < 0 || dev >= kMaxDev) return fail(FA_ERR_UNSUPPORTED, "device index %d out of range", dev);
-  std::lock_guard<std::mutex> lock(mu);
-  if (cached[dev] == nullptr) {
-    void *ptr = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&ptr, g_splitkv_scratch);
-    if (e != cudaSuccess || ptr == nullptr)
-      return fail(FA_ERR_CUDA, "looking up the static split-KV scratch: %s", cudaGetErrorString(e));
-    cached[dev] = ptr;
-  }
-  *addr = cached[dev];
-  return FA_OK;
+  static void *cache[kMaxDev] = {nullptr};
+  return symbol_address(g_splitkv_scratch, dev, cache, mu, addr, "the static split-KV scratch");
 }
 
 }  // namespace
@@ -716,17 +764,13 @@ extern "C" fa_status fa_fwd_splitkv_static(const void *q, const void *k, const v
                                            int rel_extent, int num_splits, void *stream) {
   g_msg[0] = 0;
   if (num_splits < 0) return fail(FA_ERR_INVALID, "num_splits must be >= 0");
+  // the scratch address belongs to the device that is current for this call
   int dev = 0;
-  if ((long long)B * Sq > 0 && Sk > 0) {
-    if (cudaGetDevice(&dev) != cudaSuccess) return fail(FA_ERR_CUDA, "cudaGetDevice failed");
-    // the split count fa_fwd_splitkv will use, and the scratch it needs
-    const int bn = splitkv_bn(D);
-    int ns = num_splits > 0 ? num_splits
-                            : fa_splitkv_default_splits(B, Sq, Sk, Hq, Hkv, D, num_sms(dev));
-    const long long tiles = ((long long)Sk + bn - 1) / bn;
-    if (ns > tiles) ns = (int)tiles;
-    if (ns < 1) ns = 1;
-    const size_t need = fa_splitkv_workspace_bytes(B, Sq, Hq, D, ns);
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(FA_ERR_CUDA, "cudaGetDevice failed");
+  if ((long long)B * Sq > 0 && Sk > 0 && Hq > 0 && Hkv > 0 && Hq % Hkv == 0 && D > 0) {
+    // the split count fa_fwd_splitkv will launch, and the scratch it needs
+    const SplitPlan sp = plan_splits(B, Sq, Sk, Hq, Hkv, D, num_splits, num_sms(dev));
+    const size_t need = fa_splitkv_workspace_bytes(B, Sq, Hq, D, sp.ns);
     if (need > (size_t)FA_SPLITKV_STATIC_SCRATCH_BYTES)
       return fail(FA_ERR_WORKSPACE,
                   "split-KV partials need %zu bytes, more than the %zu-byte static scratch "

@@ -48,7 +48,8 @@
 // for each, a MODS kernel that adds the left window bound and the soft-cap.
 //
 // Every wait is bounded (see mbar_wait); a role that gives up records the
-// timeout in g_fa_error, drains what it has in flight, and leaves its loops.
+// timeout in the error word (FwdParams::err), drains what it has in flight,
+// and leaves its loops.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -56,8 +57,6 @@
 #include "sm100_ptx.cuh"
 
 namespace fab {
-
-__device__ unsigned g_fa_error;  // watchdog word, read by fa_check_device_error
 
 constexpr int kBM = 128;  // rows per Q tile = TMEM lanes
 
@@ -145,7 +144,8 @@ struct FwdParams {
   int d_out;         // head dim of the tensors (the kernel's D, or less with zero padding)
   int st32;          // 1: output rows are 32-byte aligned (32-byte stores in the epilogue)
   int B, Sq, Sk, Hq, Hkv, G, P, lgP, n_groups;
-  int total_q;
+  int total_q, total_k;
+  int max_q;         // longest q length the launch is sized for (max_seqlen_q, or Sq)
   int n_mblk;        // CTA tiles per (batch, head group, split)
   int num_splits;
   int split_keys;    // keys per split (multiple of BN); >= any k_len when 1 split
@@ -163,6 +163,9 @@ struct FwdParams {
   float inv_scale;   // 1 / softmax_scale (bias is folded into raw-score units)
   float thr_raw;     // rescale threshold 8 (log2 units) in raw-score units
   unsigned long long timeout_ns;
+  // the library's device error word (timeouts, broken input contracts);
+  // fa_check_device_error reads and clears it
+  unsigned *err;
 };
 
 // One work unit: NQ Q tiles of one (batch, head group) and one key split.
@@ -194,11 +197,47 @@ __device__ __forceinline__ int seq_tiles(const FwdParams &p, int b, int rows_per
   return ql <= 0 ? 0 : (int)(((long long)ql * p.P + rows_per_unit - 1) / rows_per_unit);
 }
 
+// Extents of sequence b: its first query token and length, its first key
+// token and the number of keys it uses.  Checks the input contract of
+// "mgoin/tml-fa4", argument contract (cu_seqlens [B+1], nondecreasing from
+// 0, last entry the total; max_seqlen_q the largest q length) and the bound
+// of seqused_k (at most the sequence's keys).  A sequence that breaks it gets
+// kErrInput recorded and `false`: its units are skipped, so nothing of it is
+// read or written out of range.
+__device__ __forceinline__ bool seq_extents(const FwdParams &p, int b, int &q_start, int &q_len,
+                                            int &k_start, int &k_len) {
+  bool ok = true;
+  if (p.cu_q != nullptr) {
+    const int q0 = __ldg(p.cu_q + b), q1 = __ldg(p.cu_q + b + 1);
+    const int k0 = __ldg(p.cu_k + b), k1 = __ldg(p.cu_k + b + 1);
+    ok = q0 >= 0 && q1 >= q0 && q1 <= p.total_q && k0 >= 0 && k1 >= k0 && k1 <= p.total_k &&
+         q1 - q0 <= p.max_q && (b != p.B - 1 || (q1 == p.total_q && k1 == p.total_k));
+    q_start = q0;
+    q_len = q1 - q0;
+    k_start = k0;
+    k_len = k1 - k0;
+  } else {
+    q_start = b * p.Sq;
+    q_len = p.Sq;
+    k_start = b * p.Sk;
+    k_len = p.Sk;
+  }
+  if (p.seqused_k != nullptr) {
+    const int su = __ldg(p.seqused_k + b);
+    ok = ok && su >= 0 && su <= k_len;
+    k_len = su;
+  }
+  if (!ok) atomicOr(p.err, kErrInput);
+  return ok;
+}
+
 // Built by one warp before the CTA's first barrier.
 template <int NQ>
 __device__ __forceinline__ void build_sched(const FwdParams &p, const Sched &sch, int lane) {
   const int B = p.B;
   for (int b = lane; b < B; b += 32) {
+    int qs, ql, ks, kl;
+    (void)seq_extents(p, b, qs, ql, ks, kl);  // records a broken contract (units are skipped later)
     const int nb = seq_tiles(p, b, NQ * kBM);
     int rank = 0;
     for (int o = 0; o < B; ++o) {
@@ -267,18 +306,7 @@ __device__ __forceinline__ bool decode_unit(const FwdParams &p, const Sched &sch
   }
   U.hq0 = grp * p.P;
   U.hk = U.hq0 / p.G;
-  if (p.cu_q != nullptr) {
-    U.q_start = __ldg(p.cu_q + U.b);
-    U.q_len = __ldg(p.cu_q + U.b + 1) - U.q_start;
-    U.k_start = __ldg(p.cu_k + U.b);
-    U.k_len = __ldg(p.cu_k + U.b + 1) - U.k_start;
-  } else {
-    U.q_start = U.b * p.Sq;
-    U.q_len = p.Sq;
-    U.k_start = U.b * p.Sk;
-    U.k_len = p.Sk;
-  }
-  if (p.seqused_k != nullptr) U.k_len = min(max(__ldg(p.seqused_k + U.b), 0), U.k_len);
+  if (!seq_extents(p, U.b, U.q_start, U.q_len, U.k_start, U.k_len)) return false;
   U.row0 = mblk * NQ * kBM;
   if (U.row0 / p.P >= U.q_len) return false;  // no row of this unit exists
   U.active = 0;
@@ -473,7 +501,7 @@ __device__ __forceinline__ bool next_unit(const FwdParams &p, uint32_t sb, uint3
                                           bool &ok, bool warp_wide) {
   const uint32_t slot = cnt % kUnitRing;
   const uint32_t full = sb + C::kBarOff + 8u * (C::bUFull + slot);
-  bool w = mbar_wait(full, (cnt / kUnitRing) & 1u, &g_fa_error, p.timeout_ns);
+  bool w = mbar_wait(full, (cnt / kUnitRing) & 1u, p.err, p.timeout_ns);
   if (warp_wide) w = __all_sync(0xffffffffu, w);
   if (!w) {
     ok = false;
@@ -493,7 +521,7 @@ __device__ __forceinline__ void role_scheduler(const FwdParams &p, const Sched &
   auto publish = [&](const Unit &U) -> bool {
     const uint32_t slot = cnt % kUnitRing;
     if (!__all_sync(0xffffffffu, mbar_wait_sleepy(sb + C::kBarOff + 8u * (C::bUEmpty + slot),
-                                                  ((cnt / kUnitRing) & 1u) ^ 1u, &g_fa_error,
+                                                  ((cnt / kUnitRing) & 1u) ^ 1u, p.err,
                                                   p.timeout_ns)))
       return false;
     if ((threadIdx.x & 31u) == 0) {  // the warp stays converged; lane 0 publishes
@@ -542,7 +570,7 @@ __device__ __forceinline__ void role_producer(const FwdParams &p, uint32_t sb) {
 #pragma unroll
     for (int t = 0; t < C::NQ; ++t) {
       if (!(U.active >> t & 1u)) continue;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bQEmpty + t), (q_cnt[t] & 1u) ^ 1u, &g_fa_error, p.timeout_ns));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bQEmpty + t), (q_cnt[t] & 1u) ^ 1u, p.err, p.timeout_ns));
       if (!ok) break;
       const int tok = U.q_start + (U.row0 + t * kBM) / p.P;
       if (leader) {
@@ -559,7 +587,7 @@ __device__ __forceinline__ void role_producer(const FwdParams &p, uint32_t sb) {
       const int tok = U.k_start + U.kv_lo + n * C::BN;
       {
         const uint32_t s = C::k_slot(k_cnt);
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKEmpty + s), C::k_par(k_cnt) ^ 1u, &g_fa_error,
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKEmpty + s), C::k_par(k_cnt) ^ 1u, p.err,
                        p.timeout_ns));
         if (!ok) break;
         if (leader) {
@@ -574,7 +602,7 @@ __device__ __forceinline__ void role_producer(const FwdParams &p, uint32_t sb) {
       }
       {
         const uint32_t s = C::v_slot(v_cnt);
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bVEmpty + s), C::v_par(v_cnt) ^ 1u, &g_fa_error,
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bVEmpty + s), C::v_par(v_cnt) ^ 1u, p.err,
                        p.timeout_ns));
         if (!ok) break;
         if (leader) {
@@ -695,7 +723,7 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
     for (int t = 0; t < C::NQ; ++t) {
       sbase[t] = s_cnt[t];
       if (!(U.active >> t & 1u)) continue;
-      ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(C::bQFull + t), q_cnt[t] & 1u, &g_fa_error, p.timeout_ns));
+      ok = ok && __all_sync(0xffffffffu, mbar_wait(bar(C::bQFull + t), q_cnt[t] & 1u, p.err, p.timeout_ns));
       ++q_cnt[t];
     }
     if (!ok) break;
@@ -703,7 +731,7 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
     const uint32_t kb = k_cnt, vb = v_cnt;
 
     // prologue: S(0) for every active tile
-    ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + C::k_slot(kb)), C::k_par(kb), &g_fa_error, p.timeout_ns));
+    ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + C::k_slot(kb)), C::k_par(kb), p.err, p.timeout_ns));
     if (!ok) break;
     tc_fence_after();
 #pragma unroll
@@ -717,7 +745,7 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
     for (int n = 0; n < nb && ok; ++n) {
       const uint32_t kn = kb + n + 1;  // K tile of block n+1
       if (C::NS == 2 && n + 1 < nb) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + C::k_slot(kn)), C::k_par(kn), &g_fa_error,
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + C::k_slot(kn)), C::k_par(kn), p.err,
                        p.timeout_ns));
         if (!ok) break;
         tc_fence_after();
@@ -735,14 +763,14 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
         // S_t(n+1) for every tile as soon as its softmax has read S_t(n)
         if (n + 1 < nb) {
           ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + C::k_slot(kn)), C::k_par(kn),
-                                                 &g_fa_error, p.timeout_ns));
+                                                 p.err, p.timeout_ns));
           if (!ok) break;
           k_next_ready = true;
 #pragma unroll
           for (int t = 0; t < C::NQ; ++t) {
             if (!(U.active >> t & 1u)) continue;
             const uint32_t g = sbase[t] + n;
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bSRead + t), g & 1u, &g_fa_error,
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bSRead + t), g & 1u, p.err,
                                                    p.timeout_ns));
             if (!ok) break;
             tc_fence_after();
@@ -753,7 +781,7 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
           tc_commit_elect(bar(C::bKEmpty + C::k_slot(kn)));
         }
       }
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bVFull + C::v_slot(vn)), C::v_par(vn), &g_fa_error,
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bVFull + C::v_slot(vn)), C::v_par(vn), p.err,
                      p.timeout_ns));
       if (!ok) break;
 #pragma unroll
@@ -761,7 +789,7 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
         if (!(U.active >> t & 1u)) continue;
         const uint32_t g = sbase[t] + n;
         if (n == 0) {
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bOEmpty + t), (u_cnt[t] & 1u) ^ 1u, &g_fa_error, p.timeout_ns));
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bOEmpty + t), (u_cnt[t] & 1u) ^ 1u, p.err, p.timeout_ns));
           if (!ok) break;
         }
         if constexpr (C::kSplitPV) {
@@ -772,22 +800,22 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
           if (C::kSplitS && more) {
             if (!k_next_ready) {
               ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + C::k_slot(kn)),
-                                                     C::k_par(kn), &g_fa_error, p.timeout_ns));
+                                                     C::k_par(kn), p.err, p.timeout_ns));
               if (!ok) break;
               k_next_ready = true;
             }
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bSRead + t), g & 1u, &g_fa_error,
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bSRead + t), g & 1u, p.err,
                                                    p.timeout_ns));
             if (!ok) break;
             tc_fence_after();
             issue_s_half(t, g + 1, C::k_slot(kn), 1);
           }
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bPHalf + t), g & 1u, &g_fa_error,
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bPHalf + t), g & 1u, p.err,
                                                  p.timeout_ns));
           if (!ok) break;
           tc_fence_after();
           issue_pv_half(t, g, C::v_slot(vn), n == 0, 0);
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bPFull + t), g & 1u, &g_fa_error,
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bPFull + t), g & 1u, p.err,
                                                  p.timeout_ns));
           if (!ok) break;
           tc_fence_after();
@@ -801,7 +829,7 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
             } else {
               if (!k_next_ready) {
                 ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + C::k_slot(kn)),
-                                                       C::k_par(kn), &g_fa_error, p.timeout_ns));
+                                                       C::k_par(kn), p.err, p.timeout_ns));
                 if (!ok) break;
                 tc_fence_after();
                 k_next_ready = true;
@@ -813,7 +841,7 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
           }
           continue;
         }
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bPFull + t * C::NS + g % C::NS), (g / C::NS) & 1u, &g_fa_error,
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bPFull + t * C::NS + g % C::NS), (g / C::NS) & 1u, p.err,
                        p.timeout_ns));
         if (!ok) break;
         tc_fence_after();
@@ -821,7 +849,7 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
         if (t == last_t) tc_commit_elect(bar(C::bVEmpty + C::v_slot(vn)));
         if (C::NS == 1 && n + 1 < nb) {
           if (t == 0) {
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + C::k_slot(kn)), C::k_par(kn), &g_fa_error,
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bKFull + C::k_slot(kn)), C::k_par(kn), p.err,
                            p.timeout_ns));
             if (!ok) break;
             tc_fence_after();
@@ -976,7 +1004,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
       auto wait_scores = [&]() -> bool {
         const bool w = __all_sync(0xffffffffu,
                                   mbar_wait(bar(C::bSFull + t * NS + buf), (g / NS) & 1u,
-                                            &g_fa_error, p.timeout_ns));
+                                            p.err, p.timeout_ns));
         tc_fence_after();
         return w;
       };
@@ -987,7 +1015,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
           if (NS == 2 || C::kSepP) {
             const uint32_t gp = g - 1;
             if (!__all_sync(0xffffffffu, mbar_wait(bar(C::bOFull + t * NS + gp % NS),
-                                                   (gp / NS) & 1u, &g_fa_error, p.timeout_ns)))
+                                                   (gp / NS) & 1u, p.err, p.timeout_ns)))
               return false;
             tc_fence_after();
           }
@@ -1007,7 +1035,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
       auto wait_prev_pv = [&]() -> bool {
         const uint32_t gp = g - 1;
         const bool w = __all_sync(0xffffffffu, mbar_wait(bar(C::bOFull + t * NS + gp % NS),
-                                                         (gp / NS) & 1u, &g_fa_error,
+                                                         (gp / NS) & 1u, p.err,
                                                          p.timeout_ns));
         tc_fence_after();
         return w;
@@ -1213,7 +1241,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
     if (nb > 0) {
       const uint32_t gl = s_cnt + nb - 1;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::bOFull + t * NS + gl % NS), (gl / NS) & 1u,
-                                             &g_fa_error, p.timeout_ns));
+                                             p.err, p.timeout_ns));
       if (!ok) break;
       tc_fence_after();
     }
@@ -1359,21 +1387,6 @@ __global__ void __launch_bounds__(C::kThreads, 1) fa_fwd_kernel(const __grid_con
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
-}
-
-// ---------------------------------------------------------------------------
-// watchdog self-test: one thread waits, bounded by timeout_ns, on a fresh
-// mbarrier that nothing ever arrives at, so the wait must give up, record the
-// timeout code in the watchdog word and return (no trap, no endless loop).
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(32) fa_watchdog_selftest_kernel(unsigned long long timeout_ns) {
-  __shared__ __align__(8) uint64_t bar;
-  if (threadIdx.x == 0) {
-    mbar_init(smem_u32(&bar), 1);
-    fence_mbar_init();
-  }
-  __syncwarp();
-  if (threadIdx.x == 0) (void)mbar_wait(smem_u32(&bar), 0u, &g_fa_error, timeout_ns);
 }
 
 // ---------------------------------------------------------------------------

@@ -75,12 +75,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Device watchdog codes (written to the library's error word).
-enum : unsigned { kErrTimeout = 1u };
+// Codes of the library's device error word (bits, OR-ed together):
+//   kErrTimeout  a bounded wait gave up;
+//   kErrInput    a sequence broke the input contract (cu_seqlens not
+//                nondecreasing within [0, total] or not ending at the totals,
+//                a sequence longer than max_seqlen_q, seqused_k outside
+//                [0, k length]); its work units were skipped.
+enum : unsigned { kErrTimeout = 1u, kErrInput = 2u };
 
 // Wait until the phase with the given parity has completed.  Bounded: after
-// `timeout_ns` of wall time, or as soon as another thread has raised the
-// error word, it records the timeout and returns false instead of spinning on.
+// `timeout_ns` of wall time, or as soon as another thread has recorded a
+// timeout in the error word, it records the timeout and returns false instead
+// of spinning on.  (An input-contract code does not stop other waits: the
+// units that broke the contract are skipped, the rest run to completion.)
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           unsigned *err, uint64_t timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -88,7 +95,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
-      if (*reinterpret_cast<volatile unsigned *>(err) != 0u) return false;
+      if (*reinterpret_cast<volatile unsigned *>(err) & kErrTimeout) return false;
       if (global_timer_ns() - t0 > timeout_ns) {
         atomicOr(err, kErrTimeout);
         return false;
@@ -108,7 +115,7 @@ __device__ __forceinline__ bool mbar_wait_sleepy(uint32_t bar, uint32_t parity, 
     __nanosleep(256);
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 15u) == 0) {
-      if (*reinterpret_cast<volatile unsigned *>(err) != 0u) return false;
+      if (*reinterpret_cast<volatile unsigned *>(err) & kErrTimeout) return false;
       if (global_timer_ns() - t0 > timeout_ns) {
         atomicOr(err, kErrTimeout);
         return false;
@@ -331,26 +338,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x for x <= 8 on the FMA and integer pipes instead of the MUFU unit:
-// x = j + f with j = round(x) (the 1.5 * 2^23 addition leaves round(x) in the
-// low mantissa bits), 2^f on [-1/2, 1/2] from a degree-3 polynomial fitted
-// here by a Remez exchange for minimal relative error (below 7.5e-5), and 2^j
-// applied by adding j to the exponent field.  Inputs below -126, -inf for a
-// masked key among them, give exactly 0, as the MUFU instruction does: a row
-// whose keys are all masked must keep a zero normaliser.
-__device__ __forceinline__ float ex2_poly(float x) {
-  const float xc = fmaxf(x, -126.f);
-  const float t = xc + 12582912.f;
-  const float j = t - 12582912.f;
-  const float f = xc - j;
-  const float p = fmaf(fmaf(fmaf(0.05517166905807796f, f, 0.24261112219322045f), f,
-                            0.6932609854606147f),
-                       f, 0.9999280735393961f);
-  const int e = __float_as_int(t) - 0x4B400000;
-  const float r = __int_as_float(__float_as_int(p) + (e << 23));
-  return x < -126.f ? 0.f : r;
-}
-
 // --- packed fp32 pairs (sm_100 f32x2 instructions: one issue slot per pair)
 __device__ __forceinline__ uint64_t f2(float lo, float hi) {
   uint64_t r;
@@ -377,10 +364,15 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// 2^x for a pair of finite x in [-126, 8] on the FMA and integer pipes, the
-// same construction as ex2_poly with the floating-point steps packed in
-// pairs.  Callers clamp: below -126 the result is 2^-126 rather than 0, so a
-// tile with masked (-inf) scores must not take this path.
+// 2^x for a pair of x <= 8 on the FMA and integer pipes instead of the MUFU
+// unit.  With xc = max(x, -126): xc = j + f, j = round(xc) (adding 1.5 * 2^23
+// leaves round(xc) in the low mantissa bits), 2^f for f in [-1/2, 1/2] from a
+// degree-3 polynomial with minimal relative error (a Remez exchange fitted
+// here; tests/ex2_poly_fit.py reproduces the four coefficients: relative
+// error 7.48e-5 in exact arithmetic, and below 8e-5 as evaluated here in
+// fp32), and 2^j applied by adding j to the exponent field.  Below -126 the
+// result is 2^-126 rather than 0, so callers keep masked (-inf) scores off
+// this path: a row whose keys are all masked must keep a zero normaliser.
 __device__ __forceinline__ void ex2_poly2(float x0, float x1, float &y0, float &y1) {
   const uint64_t xc = f2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
   const uint64_t t = fadd2(xc, f2(12582912.f, 12582912.f));

@@ -73,7 +73,9 @@ typedef enum {
   FA_ERR_UNSUPPORTED = 2,    /* well-formed but not served (e.g. D = 100)   */
   FA_ERR_CUDA = 3,           /* a CUDA runtime call or launch failed         */
   FA_ERR_WORKSPACE = 4,      /* split-KV workspace missing or too small      */
-  FA_ERR_DEVICE_TIMEOUT = 5  /* a kernel gave up waiting (see below)         */
+  FA_ERR_DEVICE_TIMEOUT = 5, /* a kernel gave up waiting (see below)         */
+  FA_ERR_DEVICE_INPUT = 6    /* a kernel found device-side input that breaks
+                                the contract (cu_seqlens, seqused_k; below)  */
 } fa_status;
 
 typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
@@ -85,7 +87,10 @@ typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
  *   causal: bottom-right aligned (key j admitted iff j <= i + k_len - Sq).
  *   seqused_k: NULL, or device int32 [B] with 0 <= seqused_k[b] <= Sk; batch
  *     entry b then uses keys [0, seqused_k[b]) of its padded K/V rows and
- *     k_len = seqused_k[b] in the causal and bias distance.
+ *     k_len = seqused_k[b] in the causal and bias distance.  The kernel checks
+ *     the bound on the device: an entry outside it is skipped (its rows of
+ *     out and lse keep their contents) and fa_check_device_error afterwards
+ *     returns FA_ERR_DEVICE_INPUT.
  *   rel_bias: NULL, or [B*Sq, Hq, rel_extent] in q's dtype (the dense form of
  *     the varlen layout, rows in q's flattened order), rel_extent % 128 == 0.
  */
@@ -101,10 +106,17 @@ fa_status fa_fwd(const void *q, const void *k, const void *v, void *out,
  *   lse [Hq, total_q] float32 (may be NULL)
  *   cu_seqlens_q, cu_seqlens_k: device int32 [B+1], nondecreasing, first 0,
  *     last total_q / total_k.
- *   max_seqlen_q: the largest q length (sizes the launch; rows of a longer
- *     sequence are not computed).  max_seqlen_k is accepted for API parity.
+ *   max_seqlen_q: the largest q length (it sizes the launch).  max_seqlen_k
+ *     is accepted for API parity.
  *   seqused_k: NULL or device int32 [B]; k_len_b = seqused_k[b] (at most the
  *     cu_seqlens_k length).
+ *   These device arrays are checked where the kernel reads them: a sequence
+ *     whose cu_seqlens entries leave [0, total] or decrease, whose q length
+ *     exceeds max_seqlen_q, whose seqused_k entry is outside [0, its k
+ *     length], or the last sequence when cu_seqlens does not end at the
+ *     totals, is skipped: nothing is read or written for it (its rows of out
+ *     and lse keep their contents), and fa_check_device_error afterwards
+ *     returns FA_ERR_DEVICE_INPUT.  The other sequences are computed.
  *   rel_bias: NULL or [total_q, Hq, rel_extent], rel_extent % 128 == 0.
  */
 fa_status fa_fwd_varlen(const void *q, const void *k, const void *v, void *out,
@@ -127,6 +139,9 @@ fa_status fa_fwd_varlen(const void *q, const void *k, const void *v, void *out,
  *   workspace: device memory of at least fa_splitkv_workspace_bytes(...)
  *     bytes, 16-byte aligned, owned by the caller; its contents on entry do
  *     not matter and are overwritten.
+ * A seqused_k entry outside [0, Sk] is reported as in fa_fwd, but here the
+ * rows of that batch entry in out and lse are unspecified (the merge reads
+ * partials that no kernel wrote).
  */
 size_t fa_splitkv_workspace_bytes(int B, int Sq, int Hq, int D, int num_splits);
 int fa_splitkv_default_splits(int B, int Sq, int Sk, int Hq, int Hkv, int D,
@@ -262,11 +277,16 @@ fa_status fa_combine_partials(const float *o_parts, const float *lse_parts,
                               fa_dtype dt, void *out, float *lse, void *stream);
 
 /*
- * Device-side watchdog.  Every wait inside the kernels is bounded; a kernel
- * that gives up records a code in a device word and returns without
- * trapping.  This call synchronises the current device, copies that word to
- * *code (0 = none) and, if clear != 0, resets it.  Returns FA_OK, or
- * FA_ERR_DEVICE_TIMEOUT when the word was set, or FA_ERR_CUDA.
+ * Device-side error word.  Every wait inside the kernels is bounded; a kernel
+ * that gives up records code 1 in a device word of the current device and
+ * returns without trapping (later waits of any kernel then give up at once,
+ * until the word is cleared).  A kernel that finds device-side input breaking
+ * the contract (cu_seqlens, seqused_k: see fa_fwd_varlen) records code 2,
+ * skips that sequence and computes the others.  This call synchronises the
+ * current device, copies the word to *code (0 = none; the codes are bits and
+ * may be OR-ed) and, if clear != 0, resets it.  Returns FA_OK,
+ * FA_ERR_DEVICE_TIMEOUT when bit 1 was set, FA_ERR_DEVICE_INPUT when only
+ * bit 2 was, or FA_ERR_CUDA.
  */
 fa_status fa_check_device_error(int *code, int clear);
 
@@ -279,6 +299,18 @@ fa_status fa_check_device_error(int *code, int clear);
  * word when asked).  Returns FA_OK once enqueued.
  */
 fa_status fa_watchdog_selftest(unsigned long long timeout_ns, void *stream);
+
+/*
+ * Self-test of the softmax's FMA-pipe exponential: y[i] = 2^x[i] computed by
+ * the polynomial routine that some of the softmax's exponentials take instead
+ * of the MUFU unit (a degree-3 minimax polynomial on [-1/2, 1/2] scaled by an
+ * exponent-field add; relative error below 8e-5 for -125 <= x <= 8, results
+ * below 2^-125 are not accurate, and x < -126 gives 2^-126).  x and y are
+ * device float arrays of n elements.  The pages have no counterpart: it
+ * exists so that a test can measure this routine's error on the GPU.
+ * Returns FA_OK once enqueued.
+ */
+fa_status fa_selftest_exp2_fma(const float *x, float *y, long long n, void *stream);
 
 /* Human-readable name of a status; never NULL. */
 const char *fa_status_string(fa_status s);

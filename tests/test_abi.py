@@ -254,7 +254,7 @@ def _kind_of_c(param: str) -> str:
     # size_t and unsigned long long are both 64-bit unsigned here (LP64),
     # and ctypes makes c_size_t and c_ulonglong one type
     return {"int": "i32", "fa_dtype": "i32", "fa_status": "i32", "float": "f32",
-            "size_t": "u64", "unsigned long long": "u64"}[base]
+            "size_t": "u64", "unsigned long long": "u64", "long long": "i64"}[base]
 
 
 def _kind_of_ctypes(t) -> str:
@@ -262,7 +262,7 @@ def _kind_of_ctypes(t) -> str:
         return "ptr"
     assert ctypes.sizeof(t) in (4, 8)
     return {ctypes.c_int: "i32", ctypes.c_float: "f32", ctypes.c_size_t: "u64",
-            ctypes.c_ulonglong: "u64"}[t]
+            ctypes.c_ulonglong: "u64", ctypes.c_longlong: "i64"}[t]
 
 
 def test_binding_signatures_match_the_header(lib):

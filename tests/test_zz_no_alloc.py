@@ -4,10 +4,12 @@ Some callers cannot call cudaMalloc (their device memory belongs to a host
 framework's allocator or a pool fixed at start-up, or they may not allocate
 after initialisation), so they cannot hand fa_fwd_splitkv a workspace.  The
 static entry point keeps its split partials in a fixed-size array inside the
-library instead.  These tests call it through the C ABI and check that its
-output matches fa_fwd_splitkv's (same kernels, caller workspace) within the
-parity gates the other tests use, on two calls in a row, and that an
-oversized problem is refused.
+library instead.  These tests call it through the C ABI and check its output
+on two calls in a row against fa_fwd_splitkv's (same kernels, caller
+workspace; bit for bit) and against the CPU fp64 oracle within the parity
+gates the other tests use; that an empty call before a real one leaves the
+real one correct (the scratch address is that of the current device); and
+that an oversized problem is refused.
 
 This file is named so that pytest collects it last.
 """
@@ -17,6 +19,7 @@ import pytest
 import torch
 
 import fa_inputs
+import oracle
 import exact_attention_forward_flash_b200 as fa
 from parity_util import compare
 
@@ -51,6 +54,32 @@ def test_static_matches_workspace_entry_twice(D, ns):
         compare(out, lse, ref_o.float().cpu().numpy(), ref_l.cpu().numpy(),
                 what=f"static D={D} ns={ns}")
         assert torch.equal(out, ref_o) and torch.equal(lse, ref_l)
+        # and against the oracle, which shares nothing with either entry point
+        ro, rl = oracle.attention(p.q, p.k, p.v, causal=True)
+        compare(out, lse, ro, rl, what=f"static D={D} ns={ns} vs oracle")
+
+
+def test_empty_call_before_a_real_one():
+    # an empty problem (no query rows, then no keys) goes first on this
+    # device; the real call after it must get this device's scratch
+    lib = fa.load_library()
+    p = fa_inputs.random_dense(777, 2, 3, 2000, 8, 2, 128)
+    g = p.to("cuda")
+    empty_q = torch.empty((0, 3, 8, 128), dtype=torch.bfloat16, device="cuda")
+    assert _static_call(lib, empty_q, g.k[:0], g.v[:0], empty_q, torch.empty(0, device="cuda"),
+                        0) == 0
+    no_k = g.k[:, :0].contiguous()
+    o0 = torch.full_like(g.q, float("nan"))
+    l0 = torch.full((2, 8, 3), float("nan"), device="cuda")
+    assert _static_call(lib, g.q, no_k, no_k, o0, l0, 0) == 0
+    torch.cuda.synchronize()
+    assert (o0 == 0).all() and torch.isneginf(l0).all()
+    out = torch.full_like(g.q, float("nan"))
+    lse = torch.full((2, 8, 3), float("nan"), device="cuda")
+    assert _static_call(lib, g.q, g.k, g.v, out, lse, 0) == 0, lib.fa_last_error_message().decode()
+    torch.cuda.synchronize()
+    ro, rl = oracle.attention(p.q, p.k, p.v)
+    compare(out, lse, ro, rl, what="static after empty calls")
 
 
 def test_static_refuses_partials_beyond_its_scratch():
