@@ -455,6 +455,46 @@ def time_short_calls(dev, n_calls: int = 2000, per_graph: int = 100, replays: in
             "fa_fwd": plain_res, "fa_fwd_splitkv": dict(split_res, num_splits=ns)}
 
 
+def time_context_parallel(dev, world: int, rank: int, local: int, dist_on: bool, steps: int,
+                          warmup: int, peaks) -> dict:
+    """The decode workload with its keys sharded across the ranks: each rank
+    holds one contiguous shard of every sequence's keys, computes its fp32
+    partial (split-KV kernel + merge into one partial), the ranks exchange the
+    partials with one NCCL all-gather, and every rank merges them in the
+    combine kernel (fa_fwd_context_parallel).  Total work is fixed as N grows
+    (strong scaling); the value is the WHOLE problem's K/V bytes over the
+    slowest rank's time.  With one rank there is no exchange."""
+    import torch
+    from exact_attention_forward_flash_b200.context_parallel import (
+        fa_fwd_context_parallel, shard_bounds)
+    full = build_problem("decode_splitkv", dev)
+    B, Sk = full.B, full.k.shape[1]
+    start, length, after = shard_bounds(Sk, world, rank)
+    k = full.k[:, start:start + length].contiguous()
+    v = full.v[:, start:start + length].contiguous()
+    q, scale, nbytes = full.q, full.softmax_scale, full.hbm_bytes()
+    del full
+    torch.cuda.empty_cache()
+    k_after = torch.full((B,), after, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, q.shape[2], q.shape[1]), dtype=torch.float32, device=dev)
+
+    def step():
+        fa_fwd_context_parallel(q, k, v, k_after=k_after, softmax_scale=scale, out=out, lse=lse)
+
+    tt, pm, ck = time_steps(step, steps, max(3, warmup), dist_on, local,
+                            label="timed steps: context parallel")
+    tt = max_over_ranks(tt, dist_on)
+    ms = tt / steps
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": DESCR["decode_splitkv"] + f", keys sharded over {world} rank(s), "
+                                                 "one NCCL all-gather of the fp32 partials",
+            "value": round(gbs, 1), "unit": "GB/s", "scaling": "strong",
+            "ms_per_step": round(ms, 4), "frac_of_peak": round(gbs / peaks["hbm_gbs"] / world, 4),
+            "keys_per_rank": length, "sm_mhz": ck.get("sm_mhz"),
+            "gpu_launches_per_step": 3, "l2": "inputs larger than L2, no flush"}
+
+
 def max_over_ranks(x: float, dist_on: bool) -> float:
     """The maximum of a per-rank time over all ranks (NCCL on the GPU, or a
     CPU tensor when the process group runs on gloo)."""
@@ -621,6 +661,13 @@ def main():
                 extras[key]["num_splits"] = r.ns
             del q, r
             torch.cuda.empty_cache()
+
+    # ---- the decode workload with its keys sharded across the ranks (the one
+    # form of the path with a data exchange between GPUs)
+    if not a.no_extras:
+        extras["decode_context_parallel"] = time_context_parallel(
+            dev, world, rank, local, dist_on, max(5, min(a.steps, 30)), a.warmup, peaks)
+        torch.cuda.empty_cache()
 
     # ---- many short calls: per-call overhead, eager and from a CUDA graph
     short = None

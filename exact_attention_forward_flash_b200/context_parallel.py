@@ -63,8 +63,11 @@ def shard_seqused(seqused_k: Sequence[int], start: int, length: int) -> Tuple[Li
 def gather_partials(o_part: torch.Tensor, lse_part: torch.Tensor,
                     group=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """All ranks' partials, stacked in rank order: ([world, rows, D],
-    [world, rows]).  One all-gather per tensor (into one buffer on NCCL)."""
+    [world, rows]).  One all-gather per tensor (into one buffer on NCCL).
+    Without an initialised process group there is one rank and no exchange."""
     import torch.distributed as dist
+    if group is None and not (dist.is_available() and dist.is_initialized()):
+        return o_part.unsqueeze(0), lse_part.unsqueeze(0)
     world = dist.get_world_size(group)
     rows, D = o_part.shape
     if dist.get_backend(group) == "nccl":

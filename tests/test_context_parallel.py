@@ -136,6 +136,101 @@ def test_two_gloo_ranks_exchange_partials_that_merge_to_the_full_result():
 
 
 # ---------------------------------------------------------------------------
+# fa_fwd_context_parallel itself over two gloo ranks, with its two device
+# steps (the shard partial, the merge) done by the oracle on CPU tensors
+# ---------------------------------------------------------------------------
+def _cp_problem():
+    g = torch.Generator().manual_seed(11)
+    B, Sq, Sk, Hq, Hkv, D, R = 2, 5, 300, 4, 2, 8, 128
+    q = torch.randn(B, Sq, Hq, D, generator=g, dtype=torch.float64)
+    k = torch.randn(B, Sk, Hkv, D, generator=g, dtype=torch.float64)
+    v = torch.randn(B, Sk, Hkv, D, generator=g, dtype=torch.float64)
+    rb = torch.randn(B, Sq, Hq, R, generator=g, dtype=torch.float64)
+    return q, k, v, rb
+
+
+def _oracle_shard_partial(q, k, v, *, k_after=None, causal=False, softmax_scale=None,
+                          seqused_k=None, rel_bias=None, window=None, softcap=0.0,
+                          num_splits=0):
+    """Stand-in for the kernel's shard partial: the oracle over a sequence
+    made of the shard's keys followed by k_after unused keys, restricted to
+    the shard (bottom-right alignment needs only the keys after the shard)."""
+    import oracle
+    after = int(k_after[0])
+    assert all(int(a) == after for a in k_after)
+    B, Sk, Hkv, D = k.shape
+    pad = torch.zeros(B, after, Hkv, D, dtype=k.dtype)
+    o, lse = oracle.attention(q.numpy(), torch.cat([k, pad], 1).numpy(),
+                              torch.cat([v, pad], 1).numpy(), causal=causal,
+                              softmax_scale=softmax_scale, rel_bias=rel_bias.numpy(),
+                              kv_range=(0, Sk))
+    return _packed(o, lse)
+
+
+def _oracle_combine(o_all, l_all, B, Sq, Hq, *, dtype=None, out=None, lse=None):
+    """Stand-in for the merge kernel: the oracle's LSE merge."""
+    import oracle
+    o, l = oracle.lse_combine(o_all.numpy(), l_all.numpy())
+    D = o.shape[1]
+    return (torch.from_numpy(o).reshape(B, Sq, Hq, D),
+            torch.from_numpy(l).reshape(B, Sq, Hq).permute(0, 2, 1).contiguous())
+
+
+def _cp_rank_main(rank, world, port, out_q):
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from exact_attention_forward_flash_b200 import context_parallel as cp
+    cp.fa_fwd_shard_partial = _oracle_shard_partial
+    cp.fa_combine_partials = _oracle_combine
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        q, k, v, rb = _cp_problem()
+        start, length, after = cp.shard_bounds(k.shape[1], world, rank)
+        k_after = torch.full((q.shape[0],), after, dtype=torch.int32)
+        o, lse = cp.fa_fwd_context_parallel(q, k[:, start:start + length].contiguous(),
+                                            v[:, start:start + length].contiguous(),
+                                            k_after=k_after, causal=True, softmax_scale=0.3,
+                                            rel_bias=rb)
+        out_q.put((rank, o.numpy(), lse.numpy()))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_run_the_context_parallel_forward():
+    import oracle
+    world = 2
+    ctx = mp.get_context("spawn")
+    q_ = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_cp_rank_main, args=(r, world, port, q_)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted((q_.get(timeout=180) for _ in procs), key=lambda t: t[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    q, k, v, rb = _cp_problem()
+    ref_o, ref_l = oracle.attention(q.numpy(), k.numpy(), v.numpy(), causal=True,
+                                    softmax_scale=0.3, rel_bias=rb.numpy())
+    for _, o, lse in res:
+        np.testing.assert_allclose(o, ref_o, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-12)
+
+
+def test_single_process_context_parallel_needs_no_process_group():
+    from exact_attention_forward_flash_b200 import context_parallel as cp
+    o = torch.arange(6.0).reshape(3, 2)
+    l = torch.zeros(3)
+    o_all, l_all = cp.gather_partials(o, l)
+    assert o_all.shape == (1, 3, 2) and torch.equal(o_all[0], o) and l_all.shape == (1, 3)
+
+
+# ---------------------------------------------------------------------------
 # property checks of the planner over random sizes
 # ---------------------------------------------------------------------------
 from hypothesis import given, settings, strategies as st  # noqa: E402
