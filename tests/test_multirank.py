@@ -86,4 +86,4 @@ def test_reference_arm_line_follows_the_contract():
     assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "TFLOP/s"
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["e2e"]["value"] == d["value"] and d["cpu_baseline"]["kind"] == "oracle"
-    assert d["config"]["workload"].startswith("varlen_gqa_bias")
+    assert d["config"]["workload"].startswith("video_dit_20480")
