@@ -39,7 +39,7 @@ if ROOT not in sys.path:
 METRIC = "attention fwd TFLOP/s & % of BF16 tensor peak; split-KV decode HBM GB/s"
 MAIN = "video_dit_20480"
 EXTRAS = ["varlen_gqa_bias", "dense_257", "encoder_d256_seqused", "decode_splitkv", "dense_d64",
-          "local_window_softcap", "tabpfn_d16", "vision_d72"]
+          "local_window_softcap", "tabpfn_d16", "vision_d72", "dense_d256"]
 # the same shapes in fp16: a bf16 / fp16 pair per shape ("FlashAttention-4
 # backend for Blackwell #1235", Benchmarking, reports a bf16 slow-down on sm_100)
 FP16_TWINS = ["video_dit_20480", "dense_d64"]
@@ -54,6 +54,7 @@ DESCR = {
     "local_window_softcap": "causal GQA 16/4 D=128 B=1 S=32768, window 4095 left, softcap 50 bf16",
     "tabpfn_d16": "dense non-causal MHA B=1 S=30000 H=8 D=16 fp16",
     "vision_d72": "dense non-causal MHA B=32 S=729 H=16 D=72 bf16",
+    "dense_d256": "dense non-causal MHA B=4 S=4096 H=8 D=256 bf16 (CTA-pair kernel)",
 }
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
 

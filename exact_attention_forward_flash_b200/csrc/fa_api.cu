@@ -400,15 +400,27 @@ fa_status run_fwd(const Common &c, cudaStream_t st) {
   unsigned *err = nullptr;
   if ((s = current_device(&dev, &err)) != FA_OK) return s;
   FwdParams p;
-  // width <= 128: two Q tiles per CTA, 128-key tiles; 256: one Q tile, 64-key tiles
+  // width <= 128: two Q tiles per CTA, 128-key tiles.  Width 256: units of
+  // two Q tiles on a CTA pair (one tile per SM) with 128-key tiles, of which
+  // each CTA loads 64 keys of K and 128 dims of V -- when there is more than
+  // one wave of pairs; a problem of at most one wave runs one Q tile per CTA
+  // with 64-key tiles, whose shorter start-up and teardown (no cluster
+  // barriers) weigh more there than the pair's faster key loop.
   const int w = kernel_width(c.D);
-  const bool wide = w == 256;
-  if ((s = fill_params(c, p, wide ? 1 : 2, wide ? 64 : 128, 1, 0x7fffffff)) != FA_OK) return s;
+  if ((s = fill_params(c, p, 2, 128, 1, 0x7fffffff)) != FA_OK) return s;
   if (p.num_units == 0) return FA_OK;
   const bool half = c.dt == FA_FP16;
   const bool mods = uses_mods(p);
   Kind kind = Kind::kThroughput;
-  if (w <= 128 && p.num_units < num_sms(dev)) {
+  if (w == 256 && p.num_units > num_sms(dev) / 2) {
+    // K is loaded in halves of 64 keys
+    const long long tk = c.varlen ? c.total_k : (long long)c.B * c.Sk;
+    if ((s = make_map(&p.tm_k, tk > 0 ? c.k : c.q, c.D, c.Hkv, tk > 0 ? tk : 1, 1, 64, half)) != FA_OK)
+      return s;
+    kind = Kind::kPair;
+  } else if (w == 256) {
+    if ((s = fill_params(c, p, 1, 64, 1, 0x7fffffff)) != FA_OK) return s;
+  } else if (p.num_units < num_sms(dev)) {
     // fewer two-tile units than SMs: one tile per CTA, twice the units
     if ((s = fill_params(c, p, 1, 128, 1, 0x7fffffff)) != FA_OK) return s;
     kind = Kind::kLatency;

@@ -125,7 +125,7 @@ __device__ __forceinline__ float row_max(const float (&s)[M]) {
     for (int k = 0; k < 4; ++k) m4[k] = fmax3(m4[k], s[OFF + c + 2 * k], s[OFF + c + 2 * k + 1]);
   return fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
 }
-constexpr int kUnitRing = 4;      // published units in flight
+constexpr int kUnitRing = 1;      // published units in flight (one: a unit is published when every role has taken the one before)
 constexpr int kUnitBytes = 64;    // one unit record in shared memory
 
 struct FwdParams {
@@ -336,9 +336,10 @@ __device__ __forceinline__ bool decode_unit(const FwdParams &p, const Sched &sch
 // The k-th unit of this CTA in a static schedule of whole rounds of gridDim.x
 // units whose direction alternates (a "snake"): with units sorted by
 // decreasing work, each CTA's heavy and light picks even out.
-__device__ __forceinline__ int unit_of(int k) {
-  const int G = static_cast<int>(gridDim.x);
-  const int c = static_cast<int>(blockIdx.x);
+__device__ __forceinline__ int unit_of(int k, int pair_shift = 0) {
+  // CTA pairs (pair_shift 1) walk the schedule together, one unit per pair
+  const int G = static_cast<int>(gridDim.x) >> pair_shift;
+  const int c = static_cast<int>(blockIdx.x) >> pair_shift;
   return k * G + ((k & 1) ? (G - 1 - c) : c);
 }
 
@@ -371,6 +372,10 @@ template <int D_, int BN_, int NQ_, int NS_, int KST_, int VST_, bool HALF_, boo
 struct FwdCfg {
   static constexpr int D = D_, BN = BN_, NQ = NQ_, NS = NS_, KST = KST_, VST = VST_;
   static constexpr bool HALF = HALF_, PARTIAL = PARTIAL_;
+  // one CTA per unit (the paired-SM configuration is FwdPairCfg); a unit
+  // holds NQ Q tiles
+  static constexpr bool k2SM = false;
+  static constexpr int kUnitTiles = NQ_;
   // score/mask modifiers beyond causal (left window bound, soft-cap): a
   // separate kernel, so that the plain one carries none of their cost
   static constexpr bool MODS = MODS_;
@@ -534,10 +539,11 @@ __device__ __forceinline__ void role_scheduler(const FwdParams &p, const Sched &
   };
   const int n_units = p.compact ? *sch.n_units : p.num_units;
   bool ok = true;
-  for (int k = 0; k * (int)gridDim.x < n_units && ok; ++k) {
-    const int u = unit_of(k);
+  constexpr int kPS = C::k2SM ? 1 : 0;
+  for (int k = 0; k * ((int)gridDim.x >> kPS) < n_units && ok; ++k) {
+    const int u = unit_of(k, kPS);
     Unit U;
-    if (u >= n_units || !decode_unit<C::NQ, C::BN>(p, sch, u, U)) continue;
+    if (u >= n_units || !decode_unit<C::kUnitTiles, C::BN>(p, sch, u, U)) continue;
     ok = publish(U);
   }
   if (ok) {
@@ -932,10 +938,21 @@ __device__ __forceinline__ void bias_apply(const uint4 (&v)[kBiasPieces], int sh
   }
 }
 
+// t: this warpgroup's Q tile among the CTA's (its tensor-memory columns and
+// barriers); trow: that tile's index among the unit's tiles (its rows).  In
+// the paired-SM kernel each CTA holds tile t = 0 of the unit's tile `trow`
+// (its rank in the pair), and the arrivals the MMA issuer waits for (P
+// ready, O free) go to the barriers of the pair's even CTA.
 template <class C>
 __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, uint32_t tmem,
-                                             int t) {
+                                             int t, int trow) {
   auto bar = [&](int i) { return sb + C::kBarOff + 8u * i; };
+  auto arrive_mma = [&](int i) {
+    if constexpr (C::k2SM)
+      mbar_arrive_cluster(mapa_cluster(bar(i), 0));
+    else
+      mbar_arrive(bar(i));
+  };
   constexpr int BN = C::BN, NS = C::NS;
   // row pitch of the output: the tensors' head dim (the kernel's D, or less:
   // the padding columns are never stored)
@@ -950,8 +967,10 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
   uint32_t ucnt = 0;
   Unit U;
   while (ok && next_unit<C>(p, sb, ucnt, U, ok, true)) {
-    if (!(U.active >> t & 1u)) continue;
-    const int row = U.row0 + t * kBM + tid;
+    // a pair computes both of its tiles' scores in every MMA: a tile without
+    // rows still takes part (its rows are invalid and never stored)
+    if (!C::k2SM && !(U.active >> trow & 1u)) continue;
+    const int row = U.row0 + trow * kBM + tid;
     const int i = row >> p.lgP;
     const int h = U.hq0 + (row & (p.P - 1));
     const bool valid = i < U.q_len;
@@ -999,7 +1018,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
       auto warp_arrive = [&](int b) {
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(b));
+        if (lane == 0) arrive_mma(b);
       };
       auto wait_scores = [&]() -> bool {
         const bool w = __all_sync(0xffffffffu,
@@ -1320,7 +1339,12 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
     if (valid && lse_ptr != nullptr) *lse_ptr = lse_v;
     if (nb > 0) {
       tc_fence_before();
-      mbar_arrive(bar(C::bOEmpty + t));
+      if constexpr (C::k2SM) {  // one arrival per warp on the even CTA's barrier
+        __syncwarp();
+        if (lane == 0) arrive_mma(C::bOEmpty + t);
+      } else {
+        mbar_arrive(bar(C::bOEmpty + t));
+      }
     }
     s_cnt += nb;
   }
@@ -1361,7 +1385,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) fa_fwd_kernel(const __grid_con
     sch.nt = sch.sorted_b + (C::kMaxSchedB + 1);
     sch.seg_start = sch.nt + (C::kMaxSchedB + 1);
   }
-  if (warp == 2 && p.compact) build_sched<C::NQ>(p, sch, lane);
+  if (warp == 2 && p.compact) build_sched<C::kUnitTiles>(p, sch, lane);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -1378,7 +1402,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) fa_fwd_kernel(const __grid_con
     }
   } else {
     if constexpr (C::kSplitRegs) regs_raise<C::kRegsSoftmax>();
-    role_softmax<C>(p, sb, tmem, warp / 4 - 1);
+    role_softmax<C>(p, sb, tmem, warp / 4 - 1, warp / 4 - 1);
   }
   __syncwarp();
   tc_fence_before();

@@ -22,10 +22,11 @@ fa_status fail(fa_status s, const char *fmt, ...);
 // Streaming multiprocessors of device dev (cached).
 int num_sms(int dev);
 
-// The three kernel shapes of a width: two Q tiles per CTA with a single S
-// buffer each (throughput), one Q tile with a double-buffered S (calls with
-// fewer two-tile units than SMs), and the split-KV partial kernel.
-enum class Kind { kThroughput, kLatency, kPartial };
+// The kernel shapes of a width: two Q tiles per CTA with a single S buffer
+// each (throughput), one Q tile with a double-buffered S (calls with fewer
+// two-tile units than SMs), the split-KV partial kernel, and (width 256) the
+// CTA-pair kernel whose units of 256 rows span two SMs.
+enum class Kind { kThroughput, kLatency, kPartial, kPair };
 
 template <class C>
 fa_status launch_fwd(FwdParams &p, int dev, cudaStream_t st) {

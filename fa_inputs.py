@@ -31,6 +31,10 @@ Workloads (shapes from the pages' validation tables and API contracts):
 * ``vision_d72``: dense non-causal MHA, B=32, S=729, H=16, D=72: the D72 MHA
   profile of "flashrt/fa4-cute-runtime" (a vision encoder; the page gives no
   shape: 27x27 patches, 16 heads, a batch of 32 images).
+* ``dense_d256``: dense non-causal MHA, B=4, S=4096, H=8, D=256: a head-dim-256
+  problem of several waves of 256-row units (the D256 path of
+  "flashrt/fa4-cute-runtime" at a size where the key loop dominates; the page
+  gives no shape).
 
 Seeds are 440410 + workload index (the seed style of the pages' benchmark).
 Values are drawn in float32 as N(0, 1) and rounded to the input dtype.
@@ -47,7 +51,7 @@ SEED_BASE = 440410
 
 WORKLOADS = ["dense_257", "varlen_gqa_bias", "video_dit_20480",
              "encoder_d256_seqused", "decode_splitkv", "dense_d64",
-             "local_window_softcap", "tabpfn_d16", "vision_d72"]
+             "local_window_softcap", "tabpfn_d16", "vision_d72", "dense_d256"]
 
 _CHUNK = 1 << 24
 
@@ -254,6 +258,13 @@ def make(name: str, dtype=torch.bfloat16, device="cpu", decode_sk: int = 131072)
                        max_seqlen_q=S, max_seqlen_k=S)
     if name == "vision_d72":
         B, S, H, D = 32, 729, 16, 72
+        q = _randn((B, S, H, D), g, dtype)
+        k = _randn((B, S, H, D), g, dtype)
+        v = _randn((B, S, H, D), g, dtype)
+        return Problem(name, "dense", q, k, v, softmax_scale=1 / math.sqrt(D),
+                       max_seqlen_q=S, max_seqlen_k=S)
+    if name == "dense_d256":
+        B, S, H, D = 4, 4096, 8, 256
         q = _randn((B, S, H, D), g, dtype)
         k = _randn((B, S, H, D), g, dtype)
         v = _randn((B, S, H, D), g, dtype)

@@ -206,7 +206,7 @@ def test_video_dit_20480_sampled():
     compare(go, gl, ro, rl, what="video_dit sampled")
 
 
-@pytest.mark.parametrize("name", ["dense_d64", "tabpfn_d16", "vision_d72"])
+@pytest.mark.parametrize("name", ["dense_d64", "tabpfn_d16", "vision_d72", "dense_d256"])
 def test_dense_workloads_full(name):
     p = fa_inputs.make(name)
     out, lse = run_dense(p)
@@ -565,3 +565,41 @@ def test_two_tile_modifier_kernel(D):
     out, lse = run_dense(p, window=(90, -1), softcap=6.0)
     ro, rl = ref_dense(p, window=(90, -1), softcap=6.0)
     compare(out, lse, ro, rl, what=f"two-tile window+softcap D{D}")
+
+
+# ---------------------------------------------------------------------------
+# head dim 256 beyond one wave of CTA pairs: the paired-SM kernel (units of
+# 256 rows over two SMs); the smaller D=256 cases above take the one-CTA one
+# ---------------------------------------------------------------------------
+PAIR_CASES = [
+    # B, Sq, Sk, Hq, Hkv, D, causal -> > 74 units of 256 packed rows
+    (2, 300, 300, 48, 48, 256, True),
+    (2, 300, 333, 64, 8, 256, False),    # 8 heads packed per K/V head
+    (2, 260, 260, 40, 40, 136, False),   # a head dim padded up to 256
+]
+
+
+@pytest.mark.parametrize("case", PAIR_CASES)
+def test_pair_kernel_dense(case):
+    B, Sq, Sk, Hq, Hkv, D, causal = case
+    p = fa_inputs.random_dense(1500 + Hq + D, B, Sq, Sk, Hq, Hkv, D, causal=causal)
+    out, lse = run_dense(p)
+    ro, rl = ref_dense(p)
+    compare(out, lse, ro, rl, what=f"pair {case}")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_pair_kernel_varlen_bias(dtype):
+    p = fa_inputs.random_varlen(1600, [300, 513, 129, 0], [300, 513, 129, 5], Hq=64, Hkv=8, D=256,
+                                dtype=dtype, causal=True, bias_extent=256)
+    out, lse = run_varlen(p)
+    ro, rl = ref_varlen(p)
+    compare(out, lse, ro, rl, what=f"pair varlen bias {dtype}")
+
+
+def test_pair_kernel_window_softcap_seqused():
+    p = fa_inputs.random_dense(1700, 2, 300, 400, 48, 48, 256, causal=True, q_std=3.0,
+                               seqused=[350, 400], pad_value=1e4)
+    out, lse = run_dense(p, window=(90, -1), softcap=6.0)
+    ro, rl = ref_dense(p, window=(90, -1), softcap=6.0)
+    compare(out, lse, ro, rl, what="pair window+softcap+seqused")
