@@ -445,9 +445,10 @@ struct FwdCfg {
   static constexpr int kThreads = 128 * (1 + NQ);
   // registers: with two softmax warpgroups the launch budget (65536 / 384
   // threads = 168 each) is re-split so that the softmax warps hold a whole
-  // score row, or half a row plus its bias window, without spilling.
+  // score row, or half a row plus its bias window, without spilling; the
+  // modifier kernels (window bounds, soft-cap) take 224 of them.
   static constexpr bool kSplitRegs = NQ == 2;
-  static constexpr uint32_t kRegsCtl = 72, kRegsSoftmax = 216;
+  static constexpr uint32_t kRegsCtl = MODS_ ? 56 : 72, kRegsSoftmax = MODS_ ? 224 : 216;
   static_assert(!kSplitRegs || 128 * kRegsCtl + 256 * kRegsSoftmax <= 384 * 168, "register split");
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kOColBase = NQ * NS * BN;
