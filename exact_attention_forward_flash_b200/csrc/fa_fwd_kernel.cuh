@@ -64,7 +64,7 @@ constexpr int kBM = 128;  // rows per Q tile = TMEM lanes
 // pipe (ex2_poly2) rather than the MUFU unit, which at D = 128 is otherwise
 // as loaded as the tensor core (one exponential per 4*D tensor-core flops).
 #ifndef FA_POLY_PAIRS
-#define FA_POLY_PAIRS 2
+#define FA_POLY_PAIRS 1
 #endif
 constexpr int kPolyPairs = FA_POLY_PAIRS;
 

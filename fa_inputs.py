@@ -180,14 +180,16 @@ class Problem:
                        dict(self.meta), tuple(self.window), self.softcap)
 
 
-def make(name: str, dtype=torch.bfloat16, device="cpu", decode_sk: int = 131072) -> Problem:
+def make(name: str, dtype=torch.bfloat16, device="cpu", decode_sk: int = 131072,
+         dit_s: int = 20480) -> Problem:
     """Build one named workload with its fixed seed.
 
     With ``device`` other than the CPU the values are drawn there by that
     device's seeded generator (another stream of numbers than the CPU
     generator's, same distributions and shapes): the benchmark uses this for
     the multi-GB workloads; parity tests draw on the CPU.  ``decode_sk``
-    shortens the decode workload's keys (for profiling a smaller case)."""
+    shortens the decode workload's keys and ``dit_s`` the video workload's
+    sequence (for profiling a smaller case)."""
     idx = WORKLOADS.index(name)
     g = torch.Generator(device=device).manual_seed(SEED_BASE + idx)
     if name == "dense_257":
@@ -212,7 +214,7 @@ def make(name: str, dtype=torch.bfloat16, device="cpu", decode_sk: int = 131072)
                        max_seqlen_q=max(lens), max_seqlen_k=max(lens),
                        meta={"lens": lens})
     if name == "video_dit_20480":
-        B, S, H, D = 1, 20480, 56, 128
+        B, S, H, D = 1, int(dit_s), 56, 128
         q = _randn((B, S, H, D), g, dtype)
         k = _randn((B, S, H, D), g, dtype)
         v = _randn((B, S, H, D), g, dtype)
