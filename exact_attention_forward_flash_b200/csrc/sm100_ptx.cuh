@@ -525,6 +525,14 @@ __device__ __forceinline__ void ex2_poly2(float x0, float x1, float &y0, float &
   y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
+// tanh(x) by the hardware approximation (one MUFU operation; relative error
+// about 2^-11 as documented for tanh.approx.f32)
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ float lg2_approx(float x) {
   float y;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
