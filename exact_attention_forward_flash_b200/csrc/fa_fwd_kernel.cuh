@@ -444,10 +444,14 @@ struct FwdCfg {
   // registers: with two softmax warpgroups the launch budget (65536 / 384
   // threads = 168 each) is re-split so that the softmax warps hold a whole
   // score row, or half a row plus its bias window, without spilling; the
-  // modifier kernels (window bounds, soft-cap) take 224 of them.
-  static constexpr bool kSplitRegs = NQ == 2;
-  static constexpr uint32_t kRegsCtl = MODS_ ? 56 : 72, kRegsSoftmax = MODS_ ? 224 : 216;
-  static_assert(!kSplitRegs || 128 * kRegsCtl + 256 * kRegsSoftmax <= 384 * 168, "register split");
+  // modifier kernels (window bounds, soft-cap) take 224 of them.  With three
+  // (65536 / 512 = 128 each) the softmax warps get 152 and work on half rows.
+  static constexpr bool kSplitRegs = NQ >= 2;
+  static constexpr uint32_t kRegsCtl = NQ == 3 ? 56 : (MODS_ ? 56 : 72),
+                            kRegsSoftmax = NQ == 3 ? 152 : (MODS_ ? 224 : 216);
+  static_assert(!kSplitRegs || 128 * kRegsCtl + 128 * NQ * kRegsSoftmax <=
+                                   kThreads * ((65536 / kThreads) & ~7),
+                "register split");
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kOColBase = NQ * NS * BN;
   static constexpr int kPColBase = kOColBase + NQ * kOStride;
@@ -722,7 +726,8 @@ __device__ __forceinline__ void role_mma(const FwdParams &p, uint32_t sb, uint32
   while (ok && next_unit<C>(p, sb, ucnt, U, ok, true)) {
     if (U.nb == 0) continue;
     const int nb = U.nb;
-    const int last_t = (U.active >> 1 & 1u) && C::NQ > 1 ? 1 : 0;
+    // the last tile with rows
+    const int last_t = C::NQ == 3 ? 31 - __clz(U.active) : ((U.active >> 1 & 1u) && C::NQ > 1 ? 1 : 0);
     uint32_t sbase[C::NQ];
 #pragma unroll
     for (int t = 0; t < C::NQ; ++t) {
@@ -994,7 +999,8 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
                 : p.lse + (p.lse_dense ? ((size_t)U.b * p.Hq + h) * p.Sq + i
                                        : (size_t)h * p.total_q + U.q_start + i);
     }
-    const bool has_bias = p.rel_bias != nullptr;
+    // the three-tile kernels serve problems without a relative bias
+    const bool has_bias = C::NQ != 3 && p.rel_bias != nullptr;
     const uint16_t *brow = nullptr;
     if (has_bias && valid) brow = p.rel_bias + orow * p.R;
     float m_ref = -INFINITY, l = 0.f;
@@ -1004,8 +1010,10 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
       const int jrel = n * BN;
       const int base = base0 - jrel;  // distance of column 0
       // does any row of this warp meet the bias band in this KV tile?
-      const bool bias_blk = __any_sync(0xffffffffu, has_bias && valid && base >= 0 &&
-                                                        base - (BN - 1) < p.R);
+      // (three-tile kernels: every tile, so that a row never holds more
+      // than half of its scores)
+      const bool bias_blk = C::NQ == 3 || __any_sync(0xffffffffu, has_bias && valid && base >= 0 &&
+                                                                      base - (BN - 1) < p.R);
       const uint32_t s_addr = tmem + lane_addr + C::s_col(t, buf);
       const uint32_t p_addr = tmem + lane_addr + C::p_col(t, buf);
       const int lim_c = lim_rel - jrel;  // columns at or past lim_c are masked
@@ -1075,7 +1083,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
           return __any_sync(0xffffffffu, brow != nullptr && lo + 63 >= 0 && lo < p.R);
         };
         uint4 bv[kBiasPieces];
-        bool bon = half_on(lo0);
+        bool bon = C::NQ != 3 && half_on(lo0);
         if (bon) bias_fetch(brow, lo0, p.R, bv);
         ok = wait_scores();
         if (!ok) break;
@@ -1102,7 +1110,7 @@ __device__ __forceinline__ void role_softmax(const FwdParams &p, uint32_t sb, ui
             if (bon) bias_apply<C::HALF>(bv, bsh, p.inv_scale, x);
             if (hf + 1 < BN / 64) {
               const int lo = lo0 - 64 * (hf + 1);
-              bon = half_on(lo);
+              bon = C::NQ != 3 && half_on(lo);
               if (bon) bias_fetch(brow, lo, p.R, bv);
             }
             if (lim_c < 64 * hf + 64 || st_c > 64 * hf) {

@@ -22,11 +22,14 @@ fa_status fail(fa_status s, const char *fmt, ...);
 // Streaming multiprocessors of device dev (cached).
 int num_sms(int dev);
 
-// The kernel shapes of a width: two Q tiles per CTA with a single S buffer
-// each (throughput), one Q tile with a double-buffered S (calls with fewer
-// two-tile units than SMs), the split-KV partial kernel, and (width 256) the
-// CTA-pair kernel whose units of 256 rows span two SMs.
-enum class Kind { kThroughput, kLatency, kPartial, kPair };
+// The kernel shapes of a width: several Q tiles per CTA with a single S
+// buffer each (throughput: two tiles, three at widths 16 and 32), one Q tile
+// with a double-buffered S (calls with fewer two-tile units than SMs), the
+// split-KV partial kernel, (width 256) the CTA-pair kernel whose units of 256
+// rows span two SMs, and two tiles per CTA where the throughput kernel takes
+// three (widths 16 and 32 with a relative bias, or when three-tile units
+// would leave more of the last wave idle).
+enum class Kind { kThroughput, kLatency, kPartial, kPair, kTwoTile };
 
 template <class C>
 fa_status launch_fwd(FwdParams &p, int dev, cudaStream_t st) {
@@ -60,7 +63,8 @@ template <template <bool, bool> class Fwd, template <bool, bool> class Lat,
           template <bool, bool> class Spl>
 fa_status launch_kind(Kind k, FwdParams &p, int dev, cudaStream_t st, bool half, bool mods) {
   switch (k) {
-    case Kind::kThroughput: return launch_variant<Fwd>(p, dev, st, half, mods);
+    case Kind::kThroughput:
+    case Kind::kTwoTile: return launch_variant<Fwd>(p, dev, st, half, mods);
     case Kind::kLatency: return launch_variant<Lat>(p, dev, st, half, mods);
     default: return launch_variant<Spl>(p, dev, st, half, mods);
   }

@@ -518,7 +518,7 @@ TWO_TILE_CASES = [
     (2, 300, 300, 48, 48, 128, True),
     (2, 300, 333, 64, 16, 64, False),
     (2, 260, 260, 40, 40, 128, False),
-    (2, 300, 300, 48, 48, 16, True),
+    (2, 300, 300, 48, 48, 16, True),   # width 16: three tiles (96 units, 1 wave)
     (2, 300, 333, 64, 16, 72, False),
     (2, 260, 260, 40, 40, 48, True),
 ]
@@ -556,6 +556,66 @@ def test_one_tile_kernel_fp16_varlen_bias(D):
     out, lse = run_varlen(p)
     ro, rl = ref_varlen(p)
     compare(out, lse, ro, rl, what=f"one-tile fp16 varlen bias D{D}")
+
+
+# ---------------------------------------------------------------------------
+# widths 16 and 32: three Q tiles per CTA when the problem has no relative
+# bias and the three-tile units fill the waves about as well (30 x waves(3)
+# <= 22 x waves(2)); two tiles with a bias or when they fill them better
+# ---------------------------------------------------------------------------
+THREE_TILE_CASES = [
+    # B, Sq, Sk, Hq, Hkv, D, causal, dtype -> units of 2 / 3 tiles (waves of 148)
+    (2, 700, 650, 32, 8, 32, False, torch.bfloat16),   # 176 / 128 (2 / 1 waves)
+    (1, 1000, 1000, 40, 40, 24, True, torch.bfloat16),  # 160 / 120 (2 / 1), width 32
+    (2, 700, 650, 32, 8, 16, True, torch.float16),     # 176 / 128 (2 / 1)
+    (1, 2000, 1800, 24, 24, 16, False, torch.float16),  # 192 / 144 (2 / 1)
+]
+
+
+@pytest.mark.parametrize("case", THREE_TILE_CASES)
+def test_three_tile_kernel(case):
+    B, Sq, Sk, Hq, Hkv, D, causal, dt = case
+    p = fa_inputs.random_dense(1500 + Sq + D, B, Sq, Sk, Hq, Hkv, D, causal=causal, dtype=dt)
+    out, lse = run_dense(p)
+    ro, rl = ref_dense(p)
+    compare(out, lse, ro, rl, what=f"three-tile {case}")
+
+
+def test_three_tile_kernel_varlen_ragged():
+    # 4 heads packed per K/V head; the launch is sized by the longest sequence
+    # (4800 packed rows: 608 two-tile, 416 three-tile units, 5 / 3 waves); a
+    # one-token sequence among them
+    p = fa_inputs.random_varlen(1600, [700, 1, 385, 1200], [650, 9, 385, 1200], Hq=32, Hkv=8,
+                                D=32, causal=True)
+    out, lse = run_varlen(p)
+    ro, rl = ref_varlen(p)
+    compare(out, lse, ro, rl, what="three-tile varlen")
+
+
+@pytest.mark.parametrize("D", [16, 32])
+def test_three_tile_modifier_kernel(D):
+    p = fa_inputs.random_dense(1700 + D, 2, 700, 700, 32, 32, D, causal=True, q_std=3.0)
+    out, lse = run_dense(p, window=(150, -1), softcap=6.0)
+    ro, rl = ref_dense(p, window=(150, -1), softcap=6.0)
+    compare(out, lse, ro, rl, what=f"three-tile window+softcap D{D}")
+
+
+def test_narrow_two_tile_kernel_with_bias():
+    # 8 heads packed per K/V head: 408 two-tile units, a relative bias -> two tiles
+    p = fa_inputs.random_varlen(1800, [300, 513, 129], [300, 513, 129], Hq=64, Hkv=8, D=32,
+                                causal=True, bias_extent=128)
+    out, lse = run_varlen(p)
+    ro, rl = ref_varlen(p)
+    compare(out, lse, ro, rl, what="narrow two-tile varlen bias")
+
+
+def test_narrow_two_tile_kernel_by_waves():
+    # 320 units of two tiles and 320 of three (S = 512): three waves either
+    # way, so the two-tile kernel runs
+    p = fa_inputs.random_dense(1900, 2, 512, 512, 80, 80, 16)
+    out, lse = run_dense(p)
+    ro, rl = ref_dense(p)
+    compare(out, lse, ro, rl, what="narrow two-tile by waves")
 
 
 @pytest.mark.parametrize("D", [64, 128])
