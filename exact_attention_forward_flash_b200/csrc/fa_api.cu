@@ -424,16 +424,17 @@ fa_status run_fwd(const Common &c, cudaStream_t st) {
     // fewer two-tile units than SMs: one tile per CTA, twice the units
     if ((s = fill_params(c, p, 1, 128, 1, 0x7fffffff)) != FA_OK) return s;
     kind = Kind::kLatency;
-  } else if (w <= 32) {
-    // Widths 16 and 32 take three Q tiles per CTA (no relative bias): each
-    // tile runs about 1.1x faster than with two, since the softmax of three
-    // tiles hides more of each other's latency; the unit count drops by a
-    // third, so the choice compares whole waves.
+  } else if (w <= 64) {
+    // Widths 16 to 64 take three Q tiles per CTA (no relative bias; 64-key
+    // tiles at 48 and 64, where three 128-key S buffers and O tiles would not
+    // fit in tensor memory): each tile runs about 1.1x faster than with two,
+    // since the softmax of three tiles hides more of each other's latency;
+    // the unit count drops by a third, so the choice compares whole waves.
     kind = Kind::kTwoTile;
     if (c.rel_bias == nullptr) {
       const long long sms = num_sms(dev), w2 = (p.num_units + sms - 1) / sms;
       FwdParams p3;
-      if ((s = fill_params(c, p3, 3, 128, 1, 0x7fffffff)) != FA_OK) return s;
+      if ((s = fill_params(c, p3, 3, w <= 32 ? 128 : 64, 1, 0x7fffffff)) != FA_OK) return s;
       const long long w3 = (p3.num_units + sms - 1) / sms;
       if (w3 * 3 * 10 <= w2 * 2 * 11) {
         p = p3;

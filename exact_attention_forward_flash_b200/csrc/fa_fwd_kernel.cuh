@@ -25,7 +25,7 @@
 //               overwrites S, V MN-major in shared memory).  Also owns the
 //               tensor-memory allocation.
 //   warp 3      idle.
-//   warps 4..   one 128-thread softmax warpgroup per Q tile; thread r owns
+//   warps 4..   one 128-thread softmax warpgroup per Q tile (two or three); thread r owns
 //               tile row r (= TMEM lane r).  Per KV tile it loads its score
 //               row from tensor memory, adds the relative bias, applies the
 //               masks, updates the running max, rescales O in tensor memory
@@ -42,7 +42,9 @@
 // zeros and the epilogue stores only the tensors' columns.
 //
 // Configurations (FwdCfg<D, BN, NQ, NS, KST, VST, HALF, PARTIAL, MODS>): two
-// Q tiles per CTA with one S buffer each (throughput), one Q tile with a
+// Q tiles per CTA with one S buffer each (throughput; three, with 64-key
+// tiles at widths 48 and 64, for problems of width <= 64 without a relative
+// bias), one Q tile with a
 // double-buffered S (latency-bound calls, D = 256, and the split-KV partial
 // kernels, which write normalised fp32 partials for the merge kernel), and,
 // for each, a MODS kernel that adds the left window bound and the soft-cap.

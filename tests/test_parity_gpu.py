@@ -559,9 +559,10 @@ def test_one_tile_kernel_fp16_varlen_bias(D):
 
 
 # ---------------------------------------------------------------------------
-# widths 16 and 32: three Q tiles per CTA when the problem has no relative
-# bias and the three-tile units fill the waves about as well (30 x waves(3)
-# <= 22 x waves(2)); two tiles with a bias or when they fill them better
+# widths 16 to 64: three Q tiles per CTA (64-key tiles at 48 and 64) when the
+# problem has no relative bias and the three-tile units fill the waves about
+# as well (30 x waves(3) <= 22 x waves(2)); two tiles with a bias or when they
+# fill them better
 # ---------------------------------------------------------------------------
 THREE_TILE_CASES = [
     # B, Sq, Sk, Hq, Hkv, D, causal, dtype -> units of 2 / 3 tiles (waves of 148)
@@ -569,6 +570,10 @@ THREE_TILE_CASES = [
     (1, 1000, 1000, 40, 40, 24, True, torch.bfloat16),  # 160 / 120 (2 / 1), width 32
     (2, 700, 650, 32, 8, 16, True, torch.float16),     # 176 / 128 (2 / 1)
     (1, 2000, 1800, 24, 24, 16, False, torch.float16),  # 192 / 144 (2 / 1)
+    (2, 700, 650, 32, 8, 64, False, torch.bfloat16),   # 176 / 128, width 64
+    (1, 1000, 1000, 40, 40, 48, True, torch.float16),   # 160 / 120, width 48
+    (1, 2000, 1800, 24, 24, 40, False, torch.bfloat16),  # 192 / 144, width 48
+    (2, 700, 650, 32, 8, 64, True, torch.float16),     # 176 / 128, width 64
 ]
 
 
@@ -581,18 +586,19 @@ def test_three_tile_kernel(case):
     compare(out, lse, ro, rl, what=f"three-tile {case}")
 
 
-def test_three_tile_kernel_varlen_ragged():
+@pytest.mark.parametrize("D", [32, 64])
+def test_three_tile_kernel_varlen_ragged(D):
     # 4 heads packed per K/V head; the launch is sized by the longest sequence
     # (4800 packed rows: 608 two-tile, 416 three-tile units, 5 / 3 waves); a
     # one-token sequence among them
-    p = fa_inputs.random_varlen(1600, [700, 1, 385, 1200], [650, 9, 385, 1200], Hq=32, Hkv=8,
-                                D=32, causal=True)
+    p = fa_inputs.random_varlen(1600 + D, [700, 1, 385, 1200], [650, 9, 385, 1200], Hq=32, Hkv=8,
+                                D=D, causal=True)
     out, lse = run_varlen(p)
     ro, rl = ref_varlen(p)
-    compare(out, lse, ro, rl, what="three-tile varlen")
+    compare(out, lse, ro, rl, what=f"three-tile varlen D{D}")
 
 
-@pytest.mark.parametrize("D", [16, 32])
+@pytest.mark.parametrize("D", [16, 32, 64])
 def test_three_tile_modifier_kernel(D):
     p = fa_inputs.random_dense(1700 + D, 2, 700, 700, 32, 32, D, causal=True, q_std=3.0)
     out, lse = run_dense(p, window=(150, -1), softcap=6.0)
@@ -600,27 +606,30 @@ def test_three_tile_modifier_kernel(D):
     compare(out, lse, ro, rl, what=f"three-tile window+softcap D{D}")
 
 
-def test_narrow_two_tile_kernel_with_bias():
+@pytest.mark.parametrize("D", [32, 64])
+def test_narrow_two_tile_kernel_with_bias(D):
     # 8 heads packed per K/V head: 408 two-tile units, a relative bias -> two tiles
-    p = fa_inputs.random_varlen(1800, [300, 513, 129], [300, 513, 129], Hq=64, Hkv=8, D=32,
+    p = fa_inputs.random_varlen(1800 + D, [300, 513, 129], [300, 513, 129], Hq=64, Hkv=8, D=D,
                                 causal=True, bias_extent=128)
     out, lse = run_varlen(p)
     ro, rl = ref_varlen(p)
-    compare(out, lse, ro, rl, what="narrow two-tile varlen bias")
+    compare(out, lse, ro, rl, what=f"narrow two-tile varlen bias D{D}")
 
 
-def test_narrow_two_tile_kernel_by_waves():
+@pytest.mark.parametrize("D", [16, 64])
+def test_narrow_two_tile_kernel_by_waves(D):
     # 320 units of two tiles and 320 of three (S = 512): three waves either
     # way, so the two-tile kernel runs
-    p = fa_inputs.random_dense(1900, 2, 512, 512, 80, 80, 16)
+    p = fa_inputs.random_dense(1900 + D, 2, 512, 512, 80, 80, D)
     out, lse = run_dense(p)
     ro, rl = ref_dense(p)
-    compare(out, lse, ro, rl, what="narrow two-tile by waves")
+    compare(out, lse, ro, rl, what=f"narrow two-tile by waves D{D}")
 
 
 @pytest.mark.parametrize("D", [64, 128])
 def test_two_tile_modifier_kernel(D):
     # >= 148 two-tile units, left window + soft-cap: the two-tile MODS kernel
+    # (at D = 64 the units fill one wave of three tiles, so that one runs)
     p = fa_inputs.random_dense(1400 + D, 2, 300, 300, 48, 48, D, causal=True, q_std=3.0)
     out, lse = run_dense(p, window=(90, -1), softcap=6.0)
     ro, rl = ref_dense(p, window=(90, -1), softcap=6.0)
