@@ -424,10 +424,10 @@ fa_status run_fwd(const Common &c, cudaStream_t st) {
     // fewer two-tile units than SMs: one tile per CTA, twice the units
     if ((s = fill_params(c, p, 1, 128, 1, 0x7fffffff)) != FA_OK) return s;
     kind = Kind::kLatency;
-  } else if (w <= 64) {
-    // Widths 16 to 64 take three Q tiles per CTA (no relative bias; 64-key
-    // tiles at 48 and 64, where three 128-key S buffers and O tiles would not
-    // fit in tensor memory): each tile runs about 1.1x faster than with two,
+  } else if (w <= 96) {
+    // Widths 16 to 96 take three Q tiles per CTA (no relative bias; 64-key
+    // tiles from width 48 up, where three 128-key S buffers and O tiles would
+    // not fit in tensor memory): each tile runs about 1.1x faster than with two,
     // since the softmax of three tiles hides more of each other's latency;
     // the unit count drops by a third, so the choice compares whole waves.
     kind = Kind::kTwoTile;

@@ -43,7 +43,7 @@
 //
 // Configurations (FwdCfg<D, BN, NQ, NS, KST, VST, HALF, PARTIAL, MODS>): two
 // Q tiles per CTA with one S buffer each (throughput; three, with 64-key
-// tiles at widths 48 and 64, for problems of width <= 64 without a relative
+// tiles from width 48 up, for problems of width <= 96 without a relative
 // bias), one Q tile with a
 // double-buffered S (latency-bound calls, D = 256, and the split-KV partial
 // kernels, which write normalised fp32 partials for the merge kernel), and,

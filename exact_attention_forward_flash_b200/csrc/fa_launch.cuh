@@ -23,11 +23,11 @@ fa_status fail(fa_status s, const char *fmt, ...);
 int num_sms(int dev);
 
 // The kernel shapes of a width: several Q tiles per CTA with a single S
-// buffer each (throughput: two tiles, three at widths 16 to 64), one Q tile
+// buffer each (throughput: two tiles, three at widths 16 to 96), one Q tile
 // with a double-buffered S (calls with fewer two-tile units than SMs), the
 // split-KV partial kernel, (width 256) the CTA-pair kernel whose units of 256
 // rows span two SMs, and two tiles per CTA where the throughput kernel takes
-// three (widths 16 to 64 with a relative bias, or when three-tile units
+// three (widths 16 to 96 with a relative bias, or when three-tile units
 // would leave more of the last wave idle).
 enum class Kind { kThroughput, kLatency, kPartial, kPair, kTwoTile };
 

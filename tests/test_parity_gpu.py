@@ -559,7 +559,7 @@ def test_one_tile_kernel_fp16_varlen_bias(D):
 
 
 # ---------------------------------------------------------------------------
-# widths 16 to 64: three Q tiles per CTA (64-key tiles at 48 and 64) when the
+# widths 16 to 96: three Q tiles per CTA (64-key tiles from 48 up) when the
 # problem has no relative bias and the three-tile units fill the waves about
 # as well (30 x waves(3) <= 22 x waves(2)); two tiles with a bias or when they
 # fill them better
@@ -574,6 +574,9 @@ THREE_TILE_CASES = [
     (1, 1000, 1000, 40, 40, 48, True, torch.float16),   # 160 / 120, width 48
     (1, 2000, 1800, 24, 24, 40, False, torch.bfloat16),  # 192 / 144, width 48
     (2, 700, 650, 32, 8, 64, True, torch.float16),     # 176 / 128, width 64
+    (2, 700, 650, 32, 8, 72, False, torch.bfloat16),   # 176 / 128, width 80
+    (1, 1000, 1000, 40, 40, 96, True, torch.float16),   # 160 / 120, width 96
+    (1, 2000, 1800, 24, 24, 88, False, torch.bfloat16),  # 192 / 144, width 96
 ]
 
 
@@ -586,7 +589,7 @@ def test_three_tile_kernel(case):
     compare(out, lse, ro, rl, what=f"three-tile {case}")
 
 
-@pytest.mark.parametrize("D", [32, 64])
+@pytest.mark.parametrize("D", [32, 64, 80])
 def test_three_tile_kernel_varlen_ragged(D):
     # 4 heads packed per K/V head; the launch is sized by the longest sequence
     # (4800 packed rows: 608 two-tile, 416 three-tile units, 5 / 3 waves); a
@@ -598,7 +601,7 @@ def test_three_tile_kernel_varlen_ragged(D):
     compare(out, lse, ro, rl, what=f"three-tile varlen D{D}")
 
 
-@pytest.mark.parametrize("D", [16, 32, 64])
+@pytest.mark.parametrize("D", [16, 32, 64, 96])
 def test_three_tile_modifier_kernel(D):
     p = fa_inputs.random_dense(1700 + D, 2, 700, 700, 32, 32, D, causal=True, q_std=3.0)
     out, lse = run_dense(p, window=(150, -1), softcap=6.0)
@@ -606,7 +609,7 @@ def test_three_tile_modifier_kernel(D):
     compare(out, lse, ro, rl, what=f"three-tile window+softcap D{D}")
 
 
-@pytest.mark.parametrize("D", [32, 64])
+@pytest.mark.parametrize("D", [32, 64, 72])
 def test_narrow_two_tile_kernel_with_bias(D):
     # 8 heads packed per K/V head: 408 two-tile units, a relative bias -> two tiles
     p = fa_inputs.random_varlen(1800 + D, [300, 513, 129], [300, 513, 129], Hq=64, Hkv=8, D=D,
@@ -616,7 +619,7 @@ def test_narrow_two_tile_kernel_with_bias(D):
     compare(out, lse, ro, rl, what=f"narrow two-tile varlen bias D{D}")
 
 
-@pytest.mark.parametrize("D", [16, 64])
+@pytest.mark.parametrize("D", [16, 64, 96])
 def test_narrow_two_tile_kernel_by_waves(D):
     # 320 units of two tiles and 320 of three (S = 512): three waves either
     # way, so the two-tile kernel runs
