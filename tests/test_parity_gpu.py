@@ -15,7 +15,7 @@ import torch
 import fa_inputs
 import oracle
 import exact_attention_forward_flash_b200 as fa
-from parity_util import compare, compare_relative, to_np
+from parity_util import compare, compare_relative
 
 pytestmark = pytest.mark.gpu
 
